@@ -1,0 +1,122 @@
+"""Bit layouts of the packed code cache, written from their documented formulas.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring). The article stores only
+the b-bit integers (Method 2); how they are packed is this library's choice,
+documented in ``include/calibq.h``. Three layouts exist; for each, this module
+maps every (token i, channel j) of one (batch, head) row to a (byte, bit)
+position and packs / unpacks with that map, one bit at a time.
+
+* canonical (any b, d*b a multiple of 32): token-major. Token i occupies
+  d*b/8 consecutive bytes; channel j's code sits at bits [j*b, j*b + b) of the
+  token's little-endian bit string, i.e. byte (j*b) // 8, bits (j*b) % 8 ...
+
+* frag-K (b = 1, d = 128): tiles of 128 tokens, 2048 bytes each. With
+  u = i % 128, grp = u >> 3, k = u & 7, g = grp & 7, wlo = grp >> 3 and
+  c = j >> 5, r = j & 31, whi = r >> 4, t = (r & 15) >> 2, ib = r & 3:
+      byte = (i // 128) * 2048 + c * 512 + (4 g + t) * 16 + (2 whi + wlo) * 4 + ib
+      bit  = k.
+
+* frag-V (b = 1, d = 128): tiles of 256 tokens, 4096 bytes each. With
+  u = i % 256, reg = u >> 7, t = (u >> 5) & 3, ib = (u >> 3) & 3, k = u & 7
+  and nb = j >> 3, g = j & 7, r = nb >> 1, e = nb & 1:
+      byte = (i // 256) * 4096 + r * 512 + (4 g + t) * 16 + (2 e + reg) * 4 + ib
+      bit  = k.
+
+Tokens past n in the last frag tile are padding and hold code 0.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+LAYOUT_CANONICAL = 0
+LAYOUT_FRAG_K = 1
+LAYOUT_FRAG_V = 2
+
+_TILE = {LAYOUT_FRAG_K: 128, LAYOUT_FRAG_V: 256}
+
+
+def _check(layout: int, d: int, bits: int):
+    if layout == LAYOUT_CANONICAL:
+        if (d * bits) % 32:
+            raise ValueError("canonical layout needs d*bits to be a multiple of 32")
+    elif layout in _TILE:
+        if bits != 1 or d != 128:
+            raise ValueError("fragment layouts are defined for bits=1, d=128")
+    else:
+        raise ValueError(f"unknown layout {layout}")
+
+
+def padded_tokens(layout: int, n: int) -> int:
+    """Tokens stored per row: n, or n rounded up to the layout's tile."""
+    if layout == LAYOUT_CANONICAL:
+        return n
+    t = _TILE[layout]
+    return -(-n // t) * t
+
+
+def codes_nbytes(layout: int, n: int, d: int, bits: int) -> int:
+    """Bytes of one (batch, head) row of packed codes."""
+    _check(layout, d, bits)
+    return padded_tokens(layout, n) * d * bits // 8
+
+
+def bit_position(layout: int, i, j, n: int, d: int, bits: int):
+    """(byte, bit) of the lowest code bit of token i, channel j within a row.
+
+    i, j may be integer arrays (broadcast together).
+    """
+    _check(layout, d, bits)
+    i = np.asarray(i, dtype=np.int64)
+    j = np.asarray(j, dtype=np.int64)
+    if layout == LAYOUT_CANONICAL:
+        row = d * bits // 8
+        pos = j * bits
+        return i * row + pos // 8, pos % 8
+    if layout == LAYOUT_FRAG_K:
+        tile, u = i // 128, i % 128
+        grp, k = u >> 3, u & 7
+        g, wlo = grp & 7, grp >> 3
+        c, r = j >> 5, j & 31
+        whi, t, ib = r >> 4, (r & 15) >> 2, r & 3
+        byte = tile * 2048 + c * 512 + (4 * g + t) * 16 + (2 * whi + wlo) * 4 + ib
+        return byte, k
+    # LAYOUT_FRAG_V
+    tile, u = i // 256, i % 256
+    reg, t, ib, k = u >> 7, (u >> 5) & 3, (u >> 3) & 3, u & 7
+    nb, g = j >> 3, j & 7
+    r, e = nb >> 1, nb & 1
+    byte = tile * 4096 + r * 512 + (4 * g + t) * 16 + (2 * e + reg) * 4 + ib
+    return byte, k
+
+
+def pack_codes(codes, layout: int, bits: int) -> np.ndarray:
+    """Pack int codes ``[B, H, n, d]`` into uint8 ``[B, H, row_bytes]``."""
+    codes = np.asarray(codes, dtype=np.int64)
+    B, H, n, d = codes.shape
+    if codes.size and (codes.min() < 0 or codes.max() > (1 << bits) - 1):
+        raise ValueError("code out of range")
+    nbytes = codes_nbytes(layout, n, d, bits)
+    ii, jj = np.meshgrid(np.arange(n), np.arange(d), indexing="ij")
+    byte, bit = bit_position(layout, ii, jj, n, d, bits)
+    # Every (token, channel) owns distinct bits, so OR-ing the shifted codes
+    # into their bytes is the same as adding them; bincount does the adding.
+    rows = np.arange(B * H, dtype=np.int64)[:, None] * nbytes
+    index = (rows + byte.ravel()[None, :]).ravel()
+    weight = (codes.reshape(B * H, n * d) << bit.ravel()[None, :]).ravel()
+    flat = np.bincount(index, weights=weight.astype(np.float64), minlength=B * H * nbytes)
+    if flat.size and flat.max() > 255:
+        raise AssertionError("two codes were mapped onto the same bits")
+    return flat.astype(np.uint8).reshape(B, H, nbytes)
+
+
+def unpack_codes(packed, layout: int, n: int, d: int, bits: int) -> np.ndarray:
+    """Inverse of ``pack_codes``: uint8 ``[B, H, row_bytes]`` -> int64 ``[B, H, n, d]``."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    B, H, nbytes = packed.shape
+    if nbytes != codes_nbytes(layout, n, d, bits):
+        raise ValueError("packed row size does not match the layout")
+    ii, jj = np.meshgrid(np.arange(n), np.arange(d), indexing="ij")
+    byte, bit = bit_position(layout, ii, jj, n, d, bits)
+    vals = packed[:, :, byte].astype(np.int64)  # [B, H, n, d]
+    return (vals >> bit) & ((1 << bits) - 1)
