@@ -1,0 +1,46 @@
+// Launchers behind the libcalibq C ABI (internal; arguments already validated).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "calibq.h"
+
+namespace cq {
+
+// ---- quantize.cu
+int quantize_splits(int rows, int n);
+size_t quantize_workspace_bytes(int rows, int n);
+cudaError_t launch_quantize(const void* x, cq_dtype dt, int rows, int n, int bits, cq_layout layout,
+                            uint8_t* codes, void* alpha, void* scale, void* workspace,
+                            cudaStream_t stream);
+
+// ---- dequant.cu
+cudaError_t launch_dequant(const uint8_t* codes, const void* alpha, const void* scale, cq_dtype dt,
+                           cq_layout layout, int rows, int n, int bits, void* out,
+                           cudaStream_t stream);
+
+// ---- decode_generic.cu (canonical layouts, any bits, any group size)
+struct DecodeArgs {
+  const void* q;
+  const uint8_t* k_codes;
+  const void* k_alpha;
+  const void* k_scale;
+  const uint8_t* v_codes;
+  const void* v_alpha;
+  const void* v_scale;
+  void* out;
+  int B, Hq, Hkv, n, bits;
+  float sigma;
+  int calib;
+  float tau_lo, tau_hi;
+};
+size_t decode_generic_workspace_bytes(int B, int Hq, int n);
+cudaError_t launch_decode_generic(const DecodeArgs& a, cq_dtype dt, void* workspace,
+                                  cudaStream_t stream);
+
+// ---- decode_frag.cu (fragment layouts, bits = 1, Hq = 4 Hkv, tensor cores)
+cudaError_t launch_decode_frag(const DecodeArgs& a, cq_dtype dt, cudaStream_t stream);
+
+}  // namespace cq

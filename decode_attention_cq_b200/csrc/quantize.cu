@@ -1,0 +1,273 @@
+// cq_quantize_kv kernels: per-channel statistics and bit packing
+// (CalibQuant article, Method 1: uniform b-bit quantization with the range
+// [alpha, beta] refined per channel over the n tokens of each (batch, head)).
+//
+// Two launches, both HBM-bound reads of the input cache:
+//   k_stats  grid (rows, S): per-split per-channel min/max -> workspace
+//   k_pack   grid (rows, tiles): folds the S partials into alpha/beta, writes
+//            alpha and the step (once per row) and the packed codes of its tile.
+#include <float.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace cq {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTpr = kD / 8;            // threads per token row (8 channels each)
+constexpr int kRpi = kThreads / kTpr;   // token rows per iteration
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_stats(const T* __restrict__ x, int n, int S,
+                                                    float* __restrict__ part) {
+  const int row = blockIdx.x, s = blockIdx.y;
+  const int per = (n + S - 1) / S;
+  const int i0 = s * per, i1 = min(n, i0 + per);
+  const int cg = threadIdx.x % kTpr, r = threadIdx.x / kTpr;
+  float mn[8], mx[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    mn[e] = FLT_MAX;
+    mx[e] = -FLT_MAX;
+  }
+  const T* base = x + (size_t)row * n * kD + cg * 8;
+  for (int i = i0 + r; i < i1; i += kRpi) {
+    float v[8];
+    load8(base + (size_t)i * kD, v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      mn[e] = fminf(mn[e], v[e]);
+      mx[e] = fmaxf(mx[e], v[e]);
+    }
+  }
+  __shared__ float smn[kRpi][kD], smx[kRpi][kD];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    smn[r][cg * 8 + e] = mn[e];
+    smx[r][cg * 8 + e] = mx[e];
+  }
+  __syncthreads();
+  if (threadIdx.x < kD) {
+    float a = FLT_MAX, b = -FLT_MAX;
+    for (int q = 0; q < kRpi; ++q) {
+      a = fminf(a, smn[q][threadIdx.x]);
+      b = fmaxf(b, smx[q][threadIdx.x]);
+    }
+    float* out = part + ((size_t)row * S + s) * 2 * kD;
+    out[threadIdx.x] = a;
+    out[kD + threadIdx.x] = b;
+  }
+}
+
+// Folds the S partials of `row` into shared alpha/beta/inv; block (row, 0)
+// also writes the stored alpha and step.
+template <typename T>
+__device__ __forceinline__ void fold_stats(const float* __restrict__ part, int row, int S, int L,
+                                           float* s_alpha, float* s_beta, float* s_inv,
+                                           T* __restrict__ alpha_out, T* __restrict__ scale_out) {
+  if (threadIdx.x < kD) {
+    const int j = threadIdx.x;
+    float a = FLT_MAX, b = -FLT_MAX;
+    const float* p = part + (size_t)row * S * 2 * kD;
+    for (int s = 0; s < S; ++s) {
+      a = fminf(a, p[s * 2 * kD + j]);
+      b = fmaxf(b, p[s * 2 * kD + kD + j]);
+    }
+    s_alpha[j] = a;
+    s_beta[j] = b;
+    s_inv[j] = (b > a) ? (float)L / (b - a) : 0.f;
+    if (blockIdx.y == 0) {
+      alpha_out[(size_t)row * kD + j] = DT<T>::from_float(a);  // exact: an input value
+      const double step = __ddiv_rn(__dsub_rn((double)b, (double)a), (double)L);
+      scale_out[(size_t)row * kD + j] = DT<T>::from_double(step);
+    }
+  }
+  __syncthreads();
+}
+
+// Canonical layout: each thread turns 8 channels of one token into 8*BITS bits.
+template <typename T, int BITS>
+__global__ void __launch_bounds__(kThreads) k_pack_canonical(
+    const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
+    uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
+  constexpr int L = (1 << BITS) - 1;
+  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
+  const int row = blockIdx.x;
+  fold_stats<T>(part, row, S, L, s_alpha, s_beta, s_inv, alpha_out, scale_out);
+  const int cg = threadIdx.x % kTpr, r = threadIdx.x / kTpr;
+  float af[8], inv[8];
+  double ad[8], bd[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    af[e] = s_alpha[cg * 8 + e];
+    inv[e] = s_inv[cg * 8 + e];
+    ad[e] = (double)af[e];
+    bd[e] = (double)s_beta[cg * 8 + e];
+  }
+  const int i0 = blockIdx.y * tile_tokens, i1 = min(n, i0 + tile_tokens);
+  const T* xr = x + (size_t)row * n * kD + cg * 8;
+  uint8_t* cr = codes + (size_t)row * n * (kD * BITS / 8) + cg * BITS;
+  for (int i = i0 + r; i < i1; i += kRpi) {
+    float v[8];
+    load8(xr + (size_t)i * kD, v);
+    uint64_t packed = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      packed |= (uint64_t)quant_code(v[e], af[e], inv[e], ad[e], bd[e], L) << (e * BITS);
+    uint8_t* dst = cr + (size_t)i * (kD * BITS / 8);
+    if (BITS == 1) *dst = (uint8_t)packed;
+    if (BITS == 2) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
+    if (BITS == 4) *reinterpret_cast<uint32_t*>(dst) = (uint32_t)packed;
+    if (BITS == 8) *reinterpret_cast<uint64_t*>(dst) = packed;
+  }
+}
+
+// FRAG_K layout (bits = 1): a thread owns one token-octet (8 tokens) x 8
+// channels, i.e. 8 bytes of the layout, written as two 32-bit words.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_pack_fragk(
+    const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
+    uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
+  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
+  const int row = blockIdx.x;
+  fold_stats<T>(part, row, S, 1, s_alpha, s_beta, s_inv, alpha_out, scale_out);
+  const int cb = threadIdx.x % kTpr, r = threadIdx.x / kTpr;
+  float af[8], inv[8];
+  double ad[8], bd[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    af[e] = s_alpha[cb * 8 + e];
+    inv[e] = s_inv[cb * 8 + e];
+    ad[e] = (double)af[e];
+    bd[e] = (double)s_beta[cb * 8 + e];
+  }
+  const int n_pad = (n + 127) / 128 * 128;
+  const int m0 = blockIdx.y * (tile_tokens / 8), m1 = min(n_pad / 8, m0 + tile_tokens / 8);
+  const T* xr = x + (size_t)row * n * kD + cb * 8;
+  uint8_t* cr = codes + (size_t)row * (n_pad / 128) * 2048;
+  // channel j = 8cb + e: c = j>>5, whi = (j&31)>>4, t = (j&15)>>2, ib = j&3
+  const int j0 = cb * 8;
+  const int c = j0 >> 5, whi = (j0 & 31) >> 4, t0 = (j0 & 15) >> 2;
+  for (int m = m0 + r; m < m1; m += kRpi) {
+    uint32_t bytes[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = 8 * m + k;
+      if (i < n) {
+        float v[8];
+        load8(xr + (size_t)i * kD, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          bytes[e] |= (uint32_t)quant_code(v[e], af[e], inv[e], ad[e], bd[e], 1) << k;
+      }
+    }
+    const int tile = m >> 4, grp = m & 15, g = grp & 7, wlo = grp >> 3;
+    uint8_t* base = cr + (size_t)tile * 2048 + c * 512 + (2 * whi + wlo) * 4;
+    const uint32_t w0 = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
+    const uint32_t w1 = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
+    *reinterpret_cast<uint32_t*>(base + (4 * g + t0) * 16) = w0;
+    *reinterpret_cast<uint32_t*>(base + (4 * g + t0 + 1) * 16) = w1;
+  }
+}
+
+// FRAG_V layout (bits = 1): a warp owns 32 consecutive tokens; lane l reads
+// token l's row and the warp ballots each channel into one 32-token word.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_pack_fragv(
+    const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
+    uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
+  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
+  const int row = blockIdx.x;
+  fold_stats<T>(part, row, S, 1, s_alpha, s_beta, s_inv, alpha_out, scale_out);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n_pad = (n + 255) / 256 * 256;
+  const int b0 = blockIdx.y * (tile_tokens / 32), b1 = min(n_pad / 32, b0 + tile_tokens / 32);
+  const T* xr = x + (size_t)row * n * kD;
+  uint8_t* cr = codes + (size_t)row * (n_pad / 256) * 4096;
+  for (int blk = b0 + warp; blk < b1; blk += kThreads / 32) {
+    const int i = blk * 32 + lane;
+    uint32_t words[4] = {0, 0, 0, 0};  // channels lane, lane+32, lane+64, lane+96
+#pragma unroll 1
+    for (int cg = 0; cg < kD / 8; ++cg) {
+      float v[8];
+      if (i < n) {
+        load8(xr + (size_t)i * kD + cg * 8, v);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int j = cg * 8 + e;
+        const int code =
+            (i < n) ? quant_code(v[e], s_alpha[j], s_inv[j], (double)s_alpha[j], (double)s_beta[j], 1)
+                    : 0;
+        const uint32_t bal = __ballot_sync(0xffffffffu, code);
+        if ((j & 31) == lane) words[j >> 5] = bal;
+      }
+    }
+    const int u = (blk * 32) & 255, tile = blk >> 3;
+    const int reg = u >> 7, t = (u >> 5) & 3;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = q * 32 + lane;
+      const int nb = j >> 3, g = j & 7, rr = nb >> 1, e = nb & 1;
+      *reinterpret_cast<uint32_t*>(cr + (size_t)tile * 4096 + rr * 512 + (4 * g + t) * 16 +
+                                   (2 * e + reg) * 4) = words[q];
+    }
+  }
+}
+
+}  // namespace
+
+int quantize_splits(int rows, int n) {
+  // Enough (row, split) blocks to fill the GPU a few times over, and at least
+  // 512 tokens per split.
+  int s = (1024 + rows - 1) / rows;
+  const int cap = (n + 511) / 512;
+  if (s > cap) s = cap;
+  return s < 1 ? 1 : s;
+}
+
+template <typename T>
+static cudaError_t launch_quantize_t(const T* x, int rows, int n, int bits, cq_layout layout,
+                                     uint8_t* codes, T* alpha, T* scale, float* part,
+                                     cudaStream_t stream) {
+  const int S = quantize_splits(rows, n);
+  k_stats<T><<<dim3(rows, S), kThreads, 0, stream>>>(x, n, S, part);
+  const int tile = 1024;
+  if (layout == CQ_LAYOUT_CANONICAL) {
+    const dim3 grid(rows, (n + tile - 1) / tile);
+    switch (bits) {
+      case 1: k_pack_canonical<T, 1><<<grid, kThreads, 0, stream>>>(x, n, S, tile, part, codes, alpha, scale); break;
+      case 2: k_pack_canonical<T, 2><<<grid, kThreads, 0, stream>>>(x, n, S, tile, part, codes, alpha, scale); break;
+      case 4: k_pack_canonical<T, 4><<<grid, kThreads, 0, stream>>>(x, n, S, tile, part, codes, alpha, scale); break;
+      default: k_pack_canonical<T, 8><<<grid, kThreads, 0, stream>>>(x, n, S, tile, part, codes, alpha, scale); break;
+    }
+  } else if (layout == CQ_LAYOUT_FRAG_K) {
+    const int n_pad = (n + 127) / 128 * 128;
+    k_pack_fragk<T><<<dim3(rows, (n_pad + tile - 1) / tile), kThreads, 0, stream>>>(
+        x, n, S, tile, part, codes, alpha, scale);
+  } else {
+    const int n_pad = (n + 255) / 256 * 256;
+    k_pack_fragv<T><<<dim3(rows, (n_pad + tile - 1) / tile), kThreads, 0, stream>>>(
+        x, n, S, tile, part, codes, alpha, scale);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const void* x, cq_dtype dt, int rows, int n, int bits, cq_layout layout,
+                            uint8_t* codes, void* alpha, void* scale, void* workspace,
+                            cudaStream_t stream) {
+  float* part = static_cast<float*>(workspace);
+  if (dt == CQ_F16)
+    return launch_quantize_t<half>(static_cast<const half*>(x), rows, n, bits, layout, codes,
+                                   static_cast<half*>(alpha), static_cast<half*>(scale), part, stream);
+  return launch_quantize_t<float>(static_cast<const float*>(x), rows, n, bits, layout, codes,
+                                  static_cast<float*>(alpha), static_cast<float*>(scale), part, stream);
+}
+
+size_t quantize_workspace_bytes(int rows, int n) {
+  return (size_t)rows * quantize_splits(rows, n) * 2 * kD * sizeof(float);
+}
+
+}  // namespace cq

@@ -1,0 +1,190 @@
+/*
+ * libcalibq -- CalibQuant's visual-KV-cache quantization and decode attention
+ * on NVIDIA B200 (sm_100a).
+ *
+ * Source of the method: the CalibQuant article (QbitAI's write-up of
+ * "CalibQuant: 1-Bit KV Cache Quantization for Multimodal LLMs", arXiv
+ * 2502.14882), sections "Method 1" (channel-wise b-bit quantization),
+ * "Method 2" (post-scaling) and "Method 3" (post-quantization calibration).
+ *
+ * Conventions shared by every entry point:
+ *
+ *  - All tensor pointers are DEVICE pointers owned by the caller (device or
+ *    managed memory of the current device; host pointers are rejected with
+ *    CQ_ERR_INVALID_ARG). The library never allocates in these calls and keeps
+ *    no mutable global state; calls are thread-safe.
+ *  - Work is enqueued asynchronously on `stream` (NULL = the legacy default
+ *    stream). A returned CQ_OK means the launch was enqueued; kernel faults
+ *    surface on the stream like any CUDA error.
+ *  - Arguments are validated on the host before anything is launched; on any
+ *    error nothing is launched and no output is written.
+ *  - Supported: head dim d = 128, bits in {1, 2, 4, 8}, n >= 1, Hq a multiple
+ *    of Hkv. Tensors are dense and contiguous (row-major, last index fastest).
+ *  - dtype CQ_F16 = IEEE binary16, CQ_F32 = IEEE binary32.
+ */
+#ifndef CALIBQ_H
+#define CALIBQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so the header needs no CUDA headers. */
+typedef struct CUstream_st* cq_stream_t;
+
+typedef enum cq_status {
+  CQ_OK = 0,
+  CQ_ERR_INVALID_ARG = 1, /* null / misaligned / host pointer, bad size, bad enum */
+  CQ_ERR_UNSUPPORTED = 2, /* valid request outside the supported set (e.g. d != 128) */
+  CQ_ERR_WORKSPACE = 3,   /* workspace missing or smaller than the *_workspace_size query */
+  CQ_ERR_CUDA = 4         /* a CUDA runtime call or launch failed */
+} cq_status;
+
+typedef enum cq_dtype { CQ_F16 = 0, CQ_F32 = 1 } cq_dtype;
+
+/*
+ * Bit layouts of a packed code row (one (batch, head) pair). A row holds the
+ * codes of tokens 0..n-1 (padded where stated); rows follow each other with no
+ * gap, so the codes buffer is [B][H][row_bytes].
+ *
+ * CQ_LAYOUT_CANONICAL (any bits; row_bytes = n * d * bits / 8):
+ *   token-major. Token i occupies d*bits/8 bytes starting at i*d*bits/8;
+ *   channel j's code is stored at bits [j*bits, j*bits+bits) of the token's
+ *   little-endian bit string, i.e. at bit (j*bits) % 32 of little-endian
+ *   uint32 word (j*bits)/32 of the token.
+ *
+ * CQ_LAYOUT_FRAG_K (bits = 1, d = 128; row_bytes = ceil(n/128) * 2048):
+ *   the K-cache layout read directly as tensor-core A fragments. Tokens form
+ *   tiles of 128 (2048 bytes each); inside a tile, token u (0..127) and
+ *   channel j map to
+ *       grp = u >> 3, k = u & 7, g = grp & 7, wlo = grp >> 3,
+ *       c = j >> 5, whi = (j & 31) >> 4, t = (j & 15) >> 2, ib = j & 3,
+ *       byte = c*512 + (4*g + t)*16 + (2*whi + wlo)*4 + ib,   bit = k.
+ *   (Each byte holds one channel of 8 consecutive tokens; lane 4g+t of a warp
+ *   loads 16 contiguous bytes per 32-channel chunk.)
+ *
+ * CQ_LAYOUT_FRAG_V (bits = 1, d = 128; row_bytes = ceil(n/256) * 4096):
+ *   the V-cache layout read directly as tensor-core B fragments. Tokens form
+ *   tiles of 256 (4096 bytes each); inside a tile, token u (0..255) and
+ *   channel j map to
+ *       reg = u >> 7, t = (u >> 5) & 3, ib = (u >> 3) & 3, k = u & 7,
+ *       nb = j >> 3, g = j & 7, r = nb >> 1, e = nb & 1,
+ *       byte = r*512 + (4*g + t)*16 + (2*e + reg)*4 + ib,     bit = k.
+ *   (Each little-endian uint32 holds 32 consecutive tokens of one channel.)
+ *
+ * Padding tokens (n..padded-1) of the fragment layouts hold code 0 and are
+ * ignored by cq_decode_attn.
+ */
+typedef enum cq_layout {
+  CQ_LAYOUT_CANONICAL = 0,
+  CQ_LAYOUT_FRAG_K = 1,
+  CQ_LAYOUT_FRAG_V = 2
+} cq_layout;
+
+/*
+ * Calibration g of the pre-softmax scores (Method 3). When enabled, every
+ * (batch, query-head) score row x with range [m, M] is mapped linearly onto
+ * [tau_lo*m, tau_hi*M]:
+ *     g(x) = tau_lo*m + (x - m) * (tau_hi*M - tau_lo*m) / (M - m),
+ * and a row with M == m is left unchanged. (The article fixes g as the linear
+ * map of the row's score range onto a target interval given by parameters;
+ * the interval [tau_lo*m, tau_hi*M] is this library's reading.) tau = (1, 1)
+ * is the identity. Requires finite tau_lo, tau_hi.
+ */
+typedef struct cq_calib {
+  int enabled;
+  float tau_lo;
+  float tau_hi;
+} cq_calib;
+
+/* Library version as 10000*major + 100*minor + patch. */
+int cq_version(void);
+
+/* Static, never-NULL description of a status code. */
+const char* cq_status_string(cq_status status);
+
+/*
+ * Bytes of a packed codes buffer [B][H][row_bytes] for the given layout.
+ * Pure host function; CQ_ERR_INVALID_ARG for bad sizes, CQ_ERR_UNSUPPORTED
+ * for a layout/bits/d combination outside the supported set.
+ */
+cq_status cq_codes_bytes(cq_layout layout, int B, int H, int n, int d, int bits, size_t* bytes);
+
+/*
+ * Workspace (device bytes, 256-byte aligned pointer) needed by cq_quantize_kv.
+ */
+cq_status cq_quantize_kv_workspace_size(int B, int H, int n, int d, size_t* bytes);
+
+/*
+ * Channel-wise b-bit quantization of one cache tensor (Method 1). Call once
+ * for K and once for V.
+ *
+ *   x       [B][H][n][d] in dtype `dt` (16-byte aligned).
+ *   codes   packed codes, cq_codes_bytes(layout, ...) bytes (16-byte aligned).
+ *   alpha   [B][H][d] in `dt`: per-channel minimum over the n tokens (exact).
+ *   scale   [B][H][d] in `dt`: per-channel step (beta - alpha) / (2^bits - 1),
+ *           computed in double and rounded once to `dt` (0 for a constant channel).
+ *   workspace / ws_bytes: at least cq_quantize_kv_workspace_size(...) bytes.
+ *
+ * Code of element x of channel j: the nearest integer to the real number
+ * (x - alpha_j) * L / (beta_j - alpha_j), L = 2^bits - 1, ties to even, taken
+ * on the IEEE double evaluation ((x - alpha) * L) / (beta - alpha); 0 when
+ * beta_j == alpha_j. (For binary16 inputs this is the exact real rounding.)
+ * The fragment layouts require bits = 1.
+ */
+cq_status cq_quantize_kv(const void* x, cq_dtype dt, int B, int H, int n, int d, int bits,
+                         cq_layout layout, uint8_t* codes, void* alpha, void* scale,
+                         void* workspace, size_t ws_bytes, cq_stream_t stream);
+
+/*
+ * Workspace needed by cq_decode_attn for this layout pair (0 for the fragment
+ * layouts, which keep every intermediate on chip).
+ */
+cq_status cq_decode_attn_workspace_size(cq_layout k_layout, cq_layout v_layout, int B, int Hq,
+                                        int Hkv, int n, int d, int bits, size_t* bytes);
+
+/*
+ * One decode step of grouped-query attention over the packed caches, with
+ * post-scaling (Method 2) and optional calibration (Method 3):
+ *
+ *   x_i = sigma * ( q . alpha_K + (q (.) s_K) . c^K_i )          (logits)
+ *   y   = g(x) if calib.enabled else x                           (per row)
+ *   p_i = exp(y_i - max y) / sum_j exp(y_j - max y)
+ *   o   = alpha_V + s_V (.) sum_i p_i c^V_i
+ *
+ * Query head h reads kv-head h / (Hq/Hkv). sigma = softmax_scale, or
+ * 1/sqrt(d) when softmax_scale == 0.
+ *
+ *   q        [B][Hq][d] in `dt`;   out [B][Hq][d] in `dt`.
+ *   k_codes/v_codes: packed as written by cq_quantize_kv with k_layout/v_layout;
+ *   k_alpha, k_scale, v_alpha, v_scale: [B][Hkv][d] in `dt`.
+ *
+ * Supported layout pairs: (CANONICAL, CANONICAL) for any bits and any Hq/Hkv;
+ * (FRAG_K, FRAG_V) for bits = 1, d = 128, Hq = 4*Hkv and n <= 65536 -- the
+ * tensor-core path.
+ */
+cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, const void* k_alpha,
+                         const void* k_scale, cq_layout k_layout, const uint8_t* v_codes,
+                         const void* v_alpha, const void* v_scale, cq_layout v_layout, int B,
+                         int Hq, int Hkv, int n, int d, int bits, float softmax_scale,
+                         cq_calib calib, void* out, void* workspace, size_t ws_bytes,
+                         cq_stream_t stream);
+
+/*
+ * Dequantize packed codes back to floating point (for checks only):
+ *   out[b][h][i][j] = alpha[b][h][j] + scale[b][h][j] * code(i, j),
+ * evaluated in double and rounded once to `dt`.
+ *   out [B][H][n][d] in `dt`.
+ */
+cq_status cq_dequant(const uint8_t* codes, const void* alpha, const void* scale, cq_dtype dt,
+                     cq_layout layout, int B, int H, int n, int d, int bits, void* out,
+                     cq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CALIBQ_H */

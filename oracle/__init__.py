@@ -45,8 +45,8 @@ from .calibquant import (  # noqa: F401
 )
 from .layouts import (  # noqa: F401
     LAYOUT_CANONICAL,
-    LAYOUT_FRAG_K,
-    LAYOUT_FRAG_V,
+    LAYOUT_OCTET_K,
+    LAYOUT_OCTET_V,
     padded_tokens,
     codes_nbytes,
     pack_codes,

@@ -10,19 +10,15 @@ position and packs / unpacks with that map, one bit at a time.
   d*b/8 consecutive bytes; channel j's code sits at bits [j*b, j*b + b) of the
   token's little-endian bit string, i.e. byte (j*b) // 8, bits (j*b) % 8 ...
 
-* frag-K (b = 1, d = 128): tiles of 128 tokens, 2048 bytes each. With
-  u = i % 128, grp = u >> 3, k = u & 7, g = grp & 7, wlo = grp >> 3 and
-  c = j >> 5, r = j & 31, whi = r >> 4, t = (r & 15) >> 2, ib = r & 3:
-      byte = (i // 128) * 2048 + c * 512 + (4 g + t) * 16 + (2 whi + wlo) * 4 + ib
-      bit  = k.
+* octet-K (b = 1, d = 128): byte-per-(8 tokens, channel). Token i,
+  channel j:   byte = (i >> 3) * 128 + j,   bit = i & 7.
+  Row bytes = ceil(n / 8) * 128.
 
-* frag-V (b = 1, d = 128): tiles of 256 tokens, 4096 bytes each. With
-  u = i % 256, reg = u >> 7, t = (u >> 5) & 3, ib = (u >> 3) & 3, k = u & 7
-  and nb = j >> 3, g = j & 7, r = nb >> 1, e = nb & 1:
-      byte = (i // 256) * 4096 + r * 512 + (4 g + t) * 16 + (2 e + reg) * 4 + ib
-      bit  = k.
+* octet-V (b = 1, d = 128): the same bytes transposed per 256-token tile.
+  Token i, channel j:   byte = (i >> 8) * 4096 + j * 32 + ((i & 255) >> 3),
+  bit = i & 7.   Row bytes = ceil(n / 256) * 4096.
 
-Tokens past n in the last frag tile are padding and hold code 0.
+Tokens past n in the last octet / tile are padding and hold code 0.
 """
 
 from __future__ import annotations
@@ -30,10 +26,10 @@ from __future__ import annotations
 import numpy as np
 
 LAYOUT_CANONICAL = 0
-LAYOUT_FRAG_K = 1
-LAYOUT_FRAG_V = 2
+LAYOUT_OCTET_K = 1
+LAYOUT_OCTET_V = 2
 
-_TILE = {LAYOUT_FRAG_K: 128, LAYOUT_FRAG_V: 256}
+_TILE = {LAYOUT_OCTET_K: 8, LAYOUT_OCTET_V: 256}
 
 
 def _check(layout: int, d: int, bits: int):
@@ -42,7 +38,7 @@ def _check(layout: int, d: int, bits: int):
             raise ValueError("canonical layout needs d*bits to be a multiple of 32")
     elif layout in _TILE:
         if bits != 1 or d != 128:
-            raise ValueError("fragment layouts are defined for bits=1, d=128")
+            raise ValueError("octet layouts are defined for bits=1, d=128")
     else:
         raise ValueError(f"unknown layout {layout}")
 
@@ -73,21 +69,10 @@ def bit_position(layout: int, i, j, n: int, d: int, bits: int):
         row = d * bits // 8
         pos = j * bits
         return i * row + pos // 8, pos % 8
-    if layout == LAYOUT_FRAG_K:
-        tile, u = i // 128, i % 128
-        grp, k = u >> 3, u & 7
-        g, wlo = grp & 7, grp >> 3
-        c, r = j >> 5, j & 31
-        whi, t, ib = r >> 4, (r & 15) >> 2, r & 3
-        byte = tile * 2048 + c * 512 + (4 * g + t) * 16 + (2 * whi + wlo) * 4 + ib
-        return byte, k
-    # LAYOUT_FRAG_V
-    tile, u = i // 256, i % 256
-    reg, t, ib, k = u >> 7, (u >> 5) & 3, (u >> 3) & 3, u & 7
-    nb, g = j >> 3, j & 7
-    r, e = nb >> 1, nb & 1
-    byte = tile * 4096 + r * 512 + (4 * g + t) * 16 + (2 * e + reg) * 4 + ib
-    return byte, k
+    if layout == LAYOUT_OCTET_K:
+        return (i >> 3) * 128 + j, i & 7
+    # LAYOUT_OCTET_V
+    return (i >> 8) * 4096 + j * 32 + ((i & 255) >> 3), i & 7
 
 
 def pack_codes(codes, layout: int, bits: int) -> np.ndarray:
