@@ -1,0 +1,369 @@
+#!/usr/bin/env python
+"""Decode-attention throughput of libcalibq on synthetic InternVL-2.5-shaped
+visual KV caches (1-bit CalibQuant: post-scaled, calibrated GQA attention over
+packed codes).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--bits B] [--path octet|canonical]
+
+One step = one decode-attention call (one layer) over a batch whose cache was
+quantized beforehand (cache fill, timed separately and reported as
+"cache_fill"). Prints ONE JSON line on rank 0. Multi-GPU runs (torchrun) give
+every rank its own batch (weak scaling, no collective on the data path); the
+step time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from decode_attention_cq_b200 import calibq as cq  # noqa: E402
+from decode_attention_cq_b200 import synth  # noqa: E402
+
+METRIC = "1-bit decode-attention tokens/s and achieved HBM GB/s (n=8192), % of roofline"
+L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
+FALLBACK_HBM_GBS = 6650.0
+CALIB = (True, 0.8, 0.9)
+DECODE_KERNEL_SOURCES = {"octet": "decode_attention_cq_b200/csrc/decode_octet.cu",
+                         "canonical": "decode_attention_cq_b200/csrc/decode_generic.cu"}
+
+
+def algorithmic_bytes(B, Hq, Hkv, n, d, bits, dsize=2):
+    """Bytes one decode step must move at least: K and V codes, per-channel
+    alpha/step of K and V, the queries and the output."""
+    codes = 2 * B * Hkv * n * d * bits // 8
+    stats = 4 * B * Hkv * d * dsize
+    qo = 2 * B * Hq * d * dsize
+    return codes + stats + qo
+
+
+def cache_fill_bytes(B, Hkv, n, d, bits, dsize=2):
+    """Reads of K and V (twice: statistics, then codes) + writes of codes/stats."""
+    x = 2 * B * Hkv * n * d * dsize
+    return 2 * x + 2 * B * Hkv * n * d * bits // 8 + 4 * B * Hkv * d * dsize
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_record(path: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel
+    source has not changed since it was captured."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(path)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, DECODE_KERNEL_SOURCES[path])
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec if rec.get("source_sha256_16") == digest else None
+
+
+class ClockSampler:
+    """Polls SM clock and throttle reasons with NVML while the timed region runs."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x1: "gpu_idle", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _poll(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(0.002)
+
+    def _sample(self):
+        if self._nv is None:
+            return
+        try:
+            self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+            r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            for bit, name in self.REASONS.items():
+                if r & bit and name != "gpu_idle":
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._poll, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self._t.join()
+        if not self.samples:
+            self._sample()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "source": "nvml, polled during the timed region"}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args, world, rank, local):
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = synth.WORKLOADS[args.workload]
+    B = args.batch or w.batch
+    n, bits = w.n, args.bits
+    layouts = ((cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V) if args.path == "octet"
+               else (cq.LAYOUT_CANONICAL, cq.LAYOUT_CANONICAL))
+    q, k, v = synth.make_case(B, w.hq, w.hkv, n, w.d, w.dtype, w.outliers, w.seed + 1000 * rank, device)
+    torch.cuda.synchronize()
+
+    # ---- cache fill (a1-a2): quantize K and V once; timed separately
+    ws = torch.empty(cq.cq_quantize_kv_workspace_size(B, w.hkv, n, w.d), dtype=torch.uint8, device=device)
+    kq = cq.cq_quantize_kv(k, bits, layouts[0], workspace=ws)
+    vq = cq.cq_quantize_kv(v, bits, layouts[1], workspace=ws)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    fill_ms = []
+    for it in range(3):
+        flush.fill_(it)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        cq.cq_quantize_kv(k, bits, layouts[0], out=kq, workspace=ws)
+        cq.cq_quantize_kv(v, bits, layouts[1], out=vq, workspace=ws)
+        e1.record(stream)
+        e1.synchronize()
+        fill_ms.append(e0.elapsed_time(e1))
+    del k, v
+    torch.cuda.empty_cache()
+
+    out = torch.empty_like(q)
+    dws_n = cq.cq_decode_attn_workspace_size(layouts[0], layouts[1], B, w.hq, w.hkv, n, w.d, bits)
+    dws = torch.empty(dws_n, dtype=torch.uint8, device=device) if dws_n else None
+    launches_per_step = 1 if args.path == "octet" else 3
+
+    def step():
+        cq.cq_decode_attn(q, kq, vq, calib=CALIB, out=out, workspace=dws)
+
+    for it in range(args.warmup):
+        flush.fill_(it & 255)
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, L2 flushed between steps (outside the events)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_wall0 = time.perf_counter()
+        for it in range(args.steps):
+            flush.fill_((it * 7) & 255)
+            starts[it].record(stream)
+            step()
+            ends[it].record(stream)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall0
+    barrier(world)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    mean_ms = max_over_ranks(sum(step_ms) / len(step_ms), world, device)
+    total_tokens = B * world  # one new token per sequence per step
+    value = total_tokens / (mean_ms * 1e-3)
+
+    # ---- end to end through the public API with host buffers
+    q_host = q.cpu().pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    q_dev = torch.empty_like(q)
+    e2e_ms = []
+    for it in range(args.warmup + args.steps):
+        flush.fill_(it & 255)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        q_dev.copy_(q_host, non_blocking=True)
+        cq.cq_decode_attn(q_dev, kq, vq, calib=CALIB, out=out, workspace=dws)
+        out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if it >= args.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_mean = max_over_ranks(sum(e2e_ms) / len(e2e_ms), world, device)
+
+    peak, peak_src = measured_peaks()
+    alg = algorithmic_bytes(B, w.hq, w.hkv, n, w.d, bits)
+    kernel_ms = sum(step_ms) / len(step_ms)  # one launch per step on the octet path
+    achieved = alg / (kernel_ms * 1e-3) / 1e9
+    trec = traffic_record(args.path)
+    fill_mean = sum(fill_ms) / len(fill_ms)
+    fill_alg = cache_fill_bytes(B, w.hkv, n, w.d, bits)
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": mean_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u1 codes, int8 tensor-core products, f32 softmax, f16 I/O" if args.path == "octet"
+        else "u%d codes, f32 math, f16 I/O" % bits,
+        "data": "synthetic (seeded InternVL-2.5-shaped K/V caches, no dataset or checkpoint)",
+        "config": {"workload": args.workload, "batch_per_gpu": B, "global_batch": B * world,
+                   "q_heads": w.hq, "kv_heads": w.hkv, "head_dim": w.d, "n_tokens": n, "bits": bits,
+                   "layout": args.path, "calibration": {"tau_lo": CALIB[1], "tau_hi": CALIB[2]},
+                   "l2": "flushed (256 MB write) between timed steps",
+                   "parallelism": f"dp{world} (independent sequences per GPU)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_src,
+                     "traffic": None if trec is None else trec["dram_bytes_per_launch"],
+                     "algorithmic_bytes_per_launch": alg,
+                     "kernel": "cq_decode_attn " + args.path},
+        "cache_fill": {"ms": fill_mean, "algorithmic_bytes": fill_alg,
+                       "achieved_gbs": fill_alg / (fill_mean * 1e-3) / 1e9},
+        "e2e": {"value": total_tokens / (e2e_mean * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": q.numel() * q.element_size(),
+                "d2h_bytes_per_step": out.numel() * out.element_size()},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+        "wall_s_timed_region": t_wall,
+    }
+    return line
+
+
+def run_oracle_sample(w, rows: int, seed: int):
+    """Times the fp64 CPU oracle's decode (given its own quantized cache) on
+    `rows` (batch, kv-head) rows of workload w; returns (seconds, rows)."""
+    import oracle
+    from oracle import calibquant as oc
+    q, k, v = synth.make_case(1, 4, 1, w.n, w.d, w.dtype, w.outliers, seed, "cpu")
+    f = lambda t: t.to(torch.float64).numpy()
+    q, k, v = f(q), f(k), f(v)
+    kq = oracle.quantize_cache(k, 1, w.dtype)
+    vq = oracle.quantize_cache(v, 1, w.dtype)
+    t0 = time.perf_counter()
+    for _ in range(rows):
+        kh = oc.dequantize(kq["codes"], kq["alpha"], kq["scale"])
+        vh = oc.dequantize(vq["codes"], vq["alpha"], vq["scale"])
+        x = oc.scores_dequantized(q, kh)
+        p = oc.softmax(oc.calibrate(x, CALIB[1], CALIB[2]))
+        oc.attend_dequantized(p, vh)
+    return time.perf_counter() - t0, rows
+
+
+def cpu_baseline(w):
+    secs, rows = run_oracle_sample(w, rows=2, seed=99)
+    seqs = rows / w.hkv  # a sequence has Hkv (batch, kv-head) rows
+    return {"value": seqs / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} (sequence, kv-head) rows of {args_global.workload} "
+                      f"(4 query heads x n={w.n} each), fp64 numpy, decode given the oracle's own "
+                      f"quantized cache; {secs:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    w = synth.WORKLOADS[args.workload]
+    times = []
+    for it in range(args.warmup + args.steps):
+        secs, rows = run_oracle_sample(w, rows=1, seed=it)
+        if it >= args.warmup:
+            times.append(secs)
+    mean = sum(times) / len(times)
+    value = (1 / w.hkv) / mean
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded InternVL-2.5-shaped K/V caches)",
+        "config": {"workload": args.workload, "bits": 1, "step": "one (sequence, kv-head) row"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"one (sequence, kv-head) row per step, n={w.n}"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+args_global = None
+
+
+def main():
+    global args_global
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="internvl8b_n8192_b64", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--batch", type=int, default=0)
+    ap.add_argument("--bits", type=int, default=1)
+    ap.add_argument("--path", choices=["octet", "canonical"], default="octet")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args_global = args
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        line = run_reference(args, world, rank)
+    else:
+        line = run_ours(args, world, rank, local)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(synth.WORKLOADS[args.workload])
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,209 @@
+// The libcalibq C ABI: host-side validation and dispatch (see include/calibq.h).
+#include <math.h>
+
+#include <limits>
+
+#include "calibq.h"
+#include "kernels.h"
+
+namespace {
+
+using cq::kD;
+
+constexpr int kVersion = 10000;  // 1.0.0
+
+bool valid_bits(int bits) { return bits == 1 || bits == 2 || bits == 4 || bits == 8; }
+bool valid_dtype(cq_dtype dt) { return dt == CQ_F16 || dt == CQ_F32; }
+bool valid_layout(cq_layout l) {
+  return l == CQ_LAYOUT_CANONICAL || l == CQ_LAYOUT_OCTET_K || l == CQ_LAYOUT_OCTET_V;
+}
+size_t dsize(cq_dtype dt) { return dt == CQ_F16 ? 2 : 4; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Device memory of the current device (or managed memory) and 16-byte aligned.
+cq_status check_ptr(const void* p) {
+  if (p == nullptr || !aligned16(p)) return CQ_ERR_INVALID_ARG;
+  cudaPointerAttributes attr;
+  cudaError_t e = cudaPointerGetAttributes(&attr, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();  // clear the sticky-free error of an unknown pointer
+    return CQ_ERR_INVALID_ARG;
+  }
+  if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+    return CQ_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CQ_ERR_CUDA;
+  if (attr.type == cudaMemoryTypeDevice && attr.device != dev) return CQ_ERR_INVALID_ARG;
+  return CQ_OK;
+}
+
+#define CQ_TRY(expr)                 \
+  do {                               \
+    const cq_status _s = (expr);     \
+    if (_s != CQ_OK) return _s;      \
+  } while (0)
+
+// Sizes shared by every entry point.
+cq_status check_shape(int B, int H, int n, int d, int bits) {
+  if (B < 1 || H < 1 || n < 1) return CQ_ERR_INVALID_ARG;
+  if (!valid_bits(bits)) return CQ_ERR_INVALID_ARG;
+  if (d != kD) return CQ_ERR_UNSUPPORTED;
+  // every element index must fit comfortably in 63 bits and rows in a grid dimension
+  if ((double)B * H * n * d > 9.0e15) return CQ_ERR_INVALID_ARG;
+  if ((long long)B * H > (long long)std::numeric_limits<int>::max()) return CQ_ERR_INVALID_ARG;
+  return CQ_OK;
+}
+
+cq_status row_bytes(cq_layout layout, int n, int bits, size_t* out) {
+  if (!valid_layout(layout)) return CQ_ERR_INVALID_ARG;
+  switch (layout) {
+    case CQ_LAYOUT_CANONICAL: *out = (size_t)n * kD * bits / 8; return CQ_OK;
+    case CQ_LAYOUT_OCTET_K:
+      if (bits != 1) return CQ_ERR_UNSUPPORTED;
+      *out = (size_t)((n + 7) / 8) * kD;
+      return CQ_OK;
+    default:
+      if (bits != 1) return CQ_ERR_UNSUPPORTED;
+      *out = (size_t)((n + 255) / 256) * 4096;
+      return CQ_OK;
+  }
+}
+
+cq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CQ_OK : CQ_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int cq_version(void) { return kVersion; }
+
+const char* cq_status_string(cq_status status) {
+  switch (status) {
+    case CQ_OK: return "CQ_OK";
+    case CQ_ERR_INVALID_ARG: return "CQ_ERR_INVALID_ARG: null, misaligned or host pointer, or a bad size/enum";
+    case CQ_ERR_UNSUPPORTED: return "CQ_ERR_UNSUPPORTED: valid request outside the supported set";
+    case CQ_ERR_WORKSPACE: return "CQ_ERR_WORKSPACE: workspace missing or too small";
+    case CQ_ERR_CUDA: return "CQ_ERR_CUDA: a CUDA call or kernel launch failed";
+  }
+  return "unknown cq_status";
+}
+
+cq_status cq_codes_bytes(cq_layout layout, int B, int H, int n, int d, int bits, size_t* bytes) {
+  if (bytes == nullptr) return CQ_ERR_INVALID_ARG;
+  CQ_TRY(check_shape(B, H, n, d, bits));
+  size_t rb = 0;
+  CQ_TRY(row_bytes(layout, n, bits, &rb));
+  *bytes = (size_t)B * H * rb;
+  return CQ_OK;
+}
+
+cq_status cq_quantize_kv_workspace_size(int B, int H, int n, int d, size_t* bytes) {
+  if (bytes == nullptr) return CQ_ERR_INVALID_ARG;
+  CQ_TRY(check_shape(B, H, n, d, 1));
+  *bytes = cq::quantize_workspace_bytes(B * H, n);
+  return CQ_OK;
+}
+
+cq_status cq_quantize_kv(const void* x, cq_dtype dt, int B, int H, int n, int d, int bits,
+                         cq_layout layout, uint8_t* codes, void* alpha, void* scale,
+                         void* workspace, size_t ws_bytes, cq_stream_t stream) {
+  if (!valid_dtype(dt)) return CQ_ERR_INVALID_ARG;
+  CQ_TRY(check_shape(B, H, n, d, bits));
+  size_t rb = 0;
+  CQ_TRY(row_bytes(layout, n, bits, &rb));
+  CQ_TRY(check_ptr(x));
+  CQ_TRY(check_ptr(codes));
+  CQ_TRY(check_ptr(alpha));
+  CQ_TRY(check_ptr(scale));
+  const size_t need = cq::quantize_workspace_bytes(B * H, n);
+  if (workspace == nullptr || ws_bytes < need) return CQ_ERR_WORKSPACE;
+  CQ_TRY(check_ptr(workspace));
+  return cuda_status(cq::launch_quantize(x, dt, B * H, n, bits, layout, codes, alpha, scale,
+                                         workspace, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+cq_status cq_decode_attn_workspace_size(cq_layout k_layout, cq_layout v_layout, int B, int Hq,
+                                        int Hkv, int n, int d, int bits, size_t* bytes) {
+  if (bytes == nullptr) return CQ_ERR_INVALID_ARG;
+  CQ_TRY(check_shape(B, Hq, n, d, bits));
+  if (Hkv < 1 || Hq % Hkv) return CQ_ERR_INVALID_ARG;
+  if (!valid_layout(k_layout) || !valid_layout(v_layout)) return CQ_ERR_INVALID_ARG;
+  if (k_layout == CQ_LAYOUT_CANONICAL && v_layout == CQ_LAYOUT_CANONICAL) {
+    *bytes = cq::decode_generic_workspace_bytes(B, Hq, n);
+    return CQ_OK;
+  }
+  if (k_layout == CQ_LAYOUT_OCTET_K && v_layout == CQ_LAYOUT_OCTET_V) {
+    *bytes = 0;
+    return CQ_OK;
+  }
+  return CQ_ERR_UNSUPPORTED;
+}
+
+cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, const void* k_alpha,
+                         const void* k_scale, cq_layout k_layout, const uint8_t* v_codes,
+                         const void* v_alpha, const void* v_scale, cq_layout v_layout, int B,
+                         int Hq, int Hkv, int n, int d, int bits, float softmax_scale,
+                         cq_calib calib, void* out, void* workspace, size_t ws_bytes,
+                         cq_stream_t stream) {
+  if (!valid_dtype(dt)) return CQ_ERR_INVALID_ARG;
+  CQ_TRY(check_shape(B, Hq, n, d, bits));
+  if (Hkv < 1 || Hq % Hkv) return CQ_ERR_INVALID_ARG;
+  if (!valid_layout(k_layout) || !valid_layout(v_layout)) return CQ_ERR_INVALID_ARG;
+  if (!isfinite(softmax_scale) || softmax_scale < 0.f) return CQ_ERR_INVALID_ARG;
+  if (calib.enabled && (!isfinite(calib.tau_lo) || !isfinite(calib.tau_hi))) return CQ_ERR_INVALID_ARG;
+  size_t rb = 0;
+  CQ_TRY(row_bytes(k_layout, n, bits, &rb));
+  CQ_TRY(row_bytes(v_layout, n, bits, &rb));
+  const bool generic = k_layout == CQ_LAYOUT_CANONICAL && v_layout == CQ_LAYOUT_CANONICAL;
+  const bool octet = k_layout == CQ_LAYOUT_OCTET_K && v_layout == CQ_LAYOUT_OCTET_V;
+  if (!generic && !octet) return CQ_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (generic && G > 32) return CQ_ERR_UNSUPPORTED;
+  if (octet && (G != 4 || bits != 1 || n > 65536)) return CQ_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k_codes, k_alpha, k_scale, v_codes, v_alpha, v_scale, out};
+  for (const void* p : ptrs) CQ_TRY(check_ptr(p));
+  cq::DecodeArgs a;
+  a.q = q;
+  a.k_codes = k_codes;
+  a.k_alpha = k_alpha;
+  a.k_scale = k_scale;
+  a.v_codes = v_codes;
+  a.v_alpha = v_alpha;
+  a.v_scale = v_scale;
+  a.out = out;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.n = n;
+  a.bits = bits;
+  a.sigma = softmax_scale == 0.f ? 1.0f / sqrtf((float)d) : softmax_scale;
+  a.calib = calib.enabled ? 1 : 0;
+  a.tau_lo = calib.tau_lo;
+  a.tau_hi = calib.tau_hi;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (generic) {
+    const size_t need = cq::decode_generic_workspace_bytes(B, Hq, n);
+    if (workspace == nullptr || ws_bytes < need) return CQ_ERR_WORKSPACE;
+    CQ_TRY(check_ptr(workspace));
+    return cuda_status(cq::launch_decode_generic(a, dt, workspace, s));
+  }
+  const cudaError_t e = cq::launch_decode_octet(a, dt, s);
+  if (e == cudaErrorNotSupported) return CQ_ERR_UNSUPPORTED;
+  return cuda_status(e);
+}
+
+cq_status cq_dequant(const uint8_t* codes, const void* alpha, const void* scale, cq_dtype dt,
+                     cq_layout layout, int B, int H, int n, int d, int bits, void* out,
+                     cq_stream_t stream) {
+  if (!valid_dtype(dt)) return CQ_ERR_INVALID_ARG;
+  CQ_TRY(check_shape(B, H, n, d, bits));
+  size_t rb = 0;
+  CQ_TRY(row_bytes(layout, n, bits, &rb));
+  if ((long long)B * H > 65535) return CQ_ERR_UNSUPPORTED;
+  const void* ptrs[] = {codes, alpha, scale, out};
+  for (const void* p : ptrs) CQ_TRY(check_ptr(p));
+  return cuda_status(cq::launch_dequant(codes, alpha, scale, dt, layout, B * H, n, bits, out,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -6,10 +6,9 @@
 #include <stdint.h>
 
 #include "calibq.h"
+#include "kernels.h"
 
 namespace cq {
-
-constexpr int kD = 128;  // head dimension supported by every kernel
 
 // ---------------------------------------------------------------- dtypes ----
 template <typename T>

@@ -10,8 +10,8 @@
 //
 // Calibration needs the range of the whole row before any weight is known,
 // hence the split. The logits go through the workspace (L2-resident for
-// moderate sizes). The tensor-core path for 1-bit fragment layouts lives in
-// decode_frag.cu.
+// moderate sizes). The tensor-core path for the 1-bit octet layouts lives in
+// decode_octet.cu.
 #include <float.h>
 
 #include "common.cuh"

@@ -9,6 +9,8 @@
 
 namespace cq {
 
+constexpr int kD = 128;  // head dimension supported by every kernel
+
 // ---- quantize.cu
 int quantize_splits(int rows, int n);
 size_t quantize_workspace_bytes(int rows, int n);
@@ -40,7 +42,7 @@ size_t decode_generic_workspace_bytes(int B, int Hq, int n);
 cudaError_t launch_decode_generic(const DecodeArgs& a, cq_dtype dt, void* workspace,
                                   cudaStream_t stream);
 
-// ---- decode_frag.cu (fragment layouts, bits = 1, Hq = 4 Hkv, tensor cores)
-cudaError_t launch_decode_frag(const DecodeArgs& a, cq_dtype dt, cudaStream_t stream);
+// ---- decode_octet.cu (octet layouts, bits = 1, Hq = 4 Hkv, tensor cores)
+cudaError_t launch_decode_octet(const DecodeArgs& a, cq_dtype dt, cudaStream_t stream);
 
 }  // namespace cq

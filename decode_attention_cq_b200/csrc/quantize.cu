@@ -124,10 +124,10 @@ __global__ void __launch_bounds__(kThreads) k_pack_canonical(
   }
 }
 
-// FRAG_K layout (bits = 1): a thread owns one token-octet (8 tokens) x 8
-// channels, i.e. 8 bytes of the layout, written as two 32-bit words.
+// OCTET_K layout (bits = 1): a thread owns one token octet (8 tokens) x 8
+// channels, i.e. 8 consecutive bytes of the layout.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) k_pack_fragk(
+__global__ void __launch_bounds__(kThreads) k_pack_octet_k(
     const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
     uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
   __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
@@ -143,15 +143,12 @@ __global__ void __launch_bounds__(kThreads) k_pack_fragk(
     ad[e] = (double)af[e];
     bd[e] = (double)s_beta[cb * 8 + e];
   }
-  const int n_pad = (n + 127) / 128 * 128;
-  const int m0 = blockIdx.y * (tile_tokens / 8), m1 = min(n_pad / 8, m0 + tile_tokens / 8);
+  const int octets = (n + 7) / 8;
+  const int m0 = blockIdx.y * (tile_tokens / 8), m1 = min(octets, m0 + tile_tokens / 8);
   const T* xr = x + (size_t)row * n * kD + cb * 8;
-  uint8_t* cr = codes + (size_t)row * (n_pad / 128) * 2048;
-  // channel j = 8cb + e: c = j>>5, whi = (j&31)>>4, t = (j&15)>>2, ib = j&3
-  const int j0 = cb * 8;
-  const int c = j0 >> 5, whi = (j0 & 31) >> 4, t0 = (j0 & 15) >> 2;
+  uint8_t* cr = codes + (size_t)row * octets * kD + cb * 8;
   for (int m = m0 + r; m < m1; m += kRpi) {
-    uint32_t bytes[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    uint64_t bytes = 0;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int i = 8 * m + k;
@@ -160,22 +157,18 @@ __global__ void __launch_bounds__(kThreads) k_pack_fragk(
         load8(xr + (size_t)i * kD, v);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          bytes[e] |= (uint32_t)quant_code(v[e], af[e], inv[e], ad[e], bd[e], 1) << k;
+          bytes |= (uint64_t)quant_code(v[e], af[e], inv[e], ad[e], bd[e], 1) << (8 * e + k);
       }
     }
-    const int tile = m >> 4, grp = m & 15, g = grp & 7, wlo = grp >> 3;
-    uint8_t* base = cr + (size_t)tile * 2048 + c * 512 + (2 * whi + wlo) * 4;
-    const uint32_t w0 = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
-    const uint32_t w1 = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
-    *reinterpret_cast<uint32_t*>(base + (4 * g + t0) * 16) = w0;
-    *reinterpret_cast<uint32_t*>(base + (4 * g + t0 + 1) * 16) = w1;
+    *reinterpret_cast<uint64_t*>(cr + (size_t)m * kD) = bytes;
   }
 }
 
-// FRAG_V layout (bits = 1): a warp owns 32 consecutive tokens; lane l reads
-// token l's row and the warp ballots each channel into one 32-token word.
+// OCTET_V layout (bits = 1): a warp owns 32 consecutive tokens; lane l reads
+// token l's row and the warp ballots each channel into one 32-token word,
+// which is bytes 4q..4q+3 of that channel's 32-byte row in the 256-token tile.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) k_pack_fragv(
+__global__ void __launch_bounds__(kThreads) k_pack_octet_v(
     const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
     uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
   __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
@@ -192,9 +185,7 @@ __global__ void __launch_bounds__(kThreads) k_pack_fragv(
 #pragma unroll 1
     for (int cg = 0; cg < kD / 8; ++cg) {
       float v[8];
-      if (i < n) {
-        load8(xr + (size_t)i * kD + cg * 8, v);
-      }
+      if (i < n) load8(xr + (size_t)i * kD + cg * 8, v);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int j = cg * 8 + e;
@@ -205,14 +196,11 @@ __global__ void __launch_bounds__(kThreads) k_pack_fragv(
         if ((j & 31) == lane) words[j >> 5] = bal;
       }
     }
-    const int u = (blk * 32) & 255, tile = blk >> 3;
-    const int reg = u >> 7, t = (u >> 5) & 3;
+    const int tile = blk >> 3, q = blk & 7;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int j = q * 32 + lane;
-      const int nb = j >> 3, g = j & 7, rr = nb >> 1, e = nb & 1;
-      *reinterpret_cast<uint32_t*>(cr + (size_t)tile * 4096 + rr * 512 + (4 * g + t) * 16 +
-                                   (2 * e + reg) * 4) = words[q];
+    for (int w = 0; w < 4; ++w) {
+      const int j = w * 32 + lane;
+      *reinterpret_cast<uint32_t*>(cr + (size_t)tile * 4096 + j * 32 + q * 4) = words[w];
     }
   }
 }
@@ -243,13 +231,13 @@ static cudaError_t launch_quantize_t(const T* x, int rows, int n, int bits, cq_l
       case 4: k_pack_canonical<T, 4><<<grid, kThreads, 0, stream>>>(x, n, S, tile, part, codes, alpha, scale); break;
       default: k_pack_canonical<T, 8><<<grid, kThreads, 0, stream>>>(x, n, S, tile, part, codes, alpha, scale); break;
     }
-  } else if (layout == CQ_LAYOUT_FRAG_K) {
-    const int n_pad = (n + 127) / 128 * 128;
-    k_pack_fragk<T><<<dim3(rows, (n_pad + tile - 1) / tile), kThreads, 0, stream>>>(
+  } else if (layout == CQ_LAYOUT_OCTET_K) {
+    const int n_pad = (n + 7) / 8 * 8;
+    k_pack_octet_k<T><<<dim3(rows, (n_pad + tile - 1) / tile), kThreads, 0, stream>>>(
         x, n, S, tile, part, codes, alpha, scale);
   } else {
     const int n_pad = (n + 255) / 256 * 256;
-    k_pack_fragv<T><<<dim3(rows, (n_pad + tile - 1) / tile), kThreads, 0, stream>>>(
+    k_pack_octet_v<T><<<dim3(rows, (n_pad + tile - 1) / tile), kThreads, 0, stream>>>(
         x, n, S, tile, part, codes, alpha, scale);
   }
   return cudaGetLastError();

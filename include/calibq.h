@@ -56,32 +56,26 @@ typedef enum cq_dtype { CQ_F16 = 0, CQ_F32 = 1 } cq_dtype;
  *   little-endian bit string, i.e. at bit (j*bits) % 32 of little-endian
  *   uint32 word (j*bits)/32 of the token.
  *
- * CQ_LAYOUT_FRAG_K (bits = 1, d = 128; row_bytes = ceil(n/128) * 2048):
- *   the K-cache layout read directly as tensor-core A fragments. Tokens form
- *   tiles of 128 (2048 bytes each); inside a tile, token u (0..127) and
- *   channel j map to
- *       grp = u >> 3, k = u & 7, g = grp & 7, wlo = grp >> 3,
- *       c = j >> 5, whi = (j & 31) >> 4, t = (j & 15) >> 2, ib = j & 3,
- *       byte = c*512 + (4*g + t)*16 + (2*whi + wlo)*4 + ib,   bit = k.
- *   (Each byte holds one channel of 8 consecutive tokens; lane 4g+t of a warp
- *   loads 16 contiguous bytes per 32-channel chunk.)
+ * CQ_LAYOUT_OCTET_K (bits = 1, d = 128; row_bytes = ceil(n/8) * 128):
+ *   one byte per (8 consecutive tokens, channel). Token i, channel j:
+ *       byte = (i >> 3) * 128 + j,        bit = i & 7.
+ *   (Row m of the [n/8][128] byte matrix is one tensor-memory lane of the
+ *   K-side tensor-core operand; masking bit k of every byte selects token
+ *   8m + k.)
  *
- * CQ_LAYOUT_FRAG_V (bits = 1, d = 128; row_bytes = ceil(n/256) * 4096):
- *   the V-cache layout read directly as tensor-core B fragments. Tokens form
- *   tiles of 256 (4096 bytes each); inside a tile, token u (0..255) and
- *   channel j map to
- *       reg = u >> 7, t = (u >> 5) & 3, ib = (u >> 3) & 3, k = u & 7,
- *       nb = j >> 3, g = j & 7, r = nb >> 1, e = nb & 1,
- *       byte = r*512 + (4*g + t)*16 + (2*e + reg)*4 + ib,     bit = k.
- *   (Each little-endian uint32 holds 32 consecutive tokens of one channel.)
+ * CQ_LAYOUT_OCTET_V (bits = 1, d = 128; row_bytes = ceil(n/256) * 4096):
+ *   the same bytes, transposed per tile of 256 tokens. Token i, channel j:
+ *       byte = (i >> 8) * 4096 + j * 32 + ((i & 255) >> 3),   bit = i & 7.
+ *   (Channel j's 32 bytes of a tile are one tensor-memory lane of the V-side
+ *   operand.)
  *
- * Padding tokens (n..padded-1) of the fragment layouts hold code 0 and are
+ * Padding tokens (n..padded-1) of the octet layouts hold code 0 and are
  * ignored by cq_decode_attn.
  */
 typedef enum cq_layout {
   CQ_LAYOUT_CANONICAL = 0,
-  CQ_LAYOUT_FRAG_K = 1,
-  CQ_LAYOUT_FRAG_V = 2
+  CQ_LAYOUT_OCTET_K = 1,
+  CQ_LAYOUT_OCTET_V = 2
 } cq_layout;
 
 /*
@@ -133,14 +127,14 @@ cq_status cq_quantize_kv_workspace_size(int B, int H, int n, int d, size_t* byte
  * (x - alpha_j) * L / (beta_j - alpha_j), L = 2^bits - 1, ties to even, taken
  * on the IEEE double evaluation ((x - alpha) * L) / (beta - alpha); 0 when
  * beta_j == alpha_j. (For binary16 inputs this is the exact real rounding.)
- * The fragment layouts require bits = 1.
+ * The octet layouts require bits = 1.
  */
 cq_status cq_quantize_kv(const void* x, cq_dtype dt, int B, int H, int n, int d, int bits,
                          cq_layout layout, uint8_t* codes, void* alpha, void* scale,
                          void* workspace, size_t ws_bytes, cq_stream_t stream);
 
 /*
- * Workspace needed by cq_decode_attn for this layout pair (0 for the fragment
+ * Workspace needed by cq_decode_attn for this layout pair (0 for the octet
  * layouts, which keep every intermediate on chip).
  */
 cq_status cq_decode_attn_workspace_size(cq_layout k_layout, cq_layout v_layout, int B, int Hq,
@@ -163,7 +157,7 @@ cq_status cq_decode_attn_workspace_size(cq_layout k_layout, cq_layout v_layout, 
  *   k_alpha, k_scale, v_alpha, v_scale: [B][Hkv][d] in `dt`.
  *
  * Supported layout pairs: (CANONICAL, CANONICAL) for any bits and any Hq/Hkv;
- * (FRAG_K, FRAG_V) for bits = 1, d = 128, Hq = 4*Hkv and n <= 65536 -- the
+ * (OCTET_K, OCTET_V) for bits = 1, d = 128, Hq = 4*Hkv and n <= 65536 -- the
  * tensor-core path.
  */
 cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, const void* k_alpha,

@@ -1,0 +1,136 @@
+"""GPU parity of the tensor-core decode path (octet layouts, 1 bit, 4 query
+heads per kv-head) against the fp64 oracle, within the 2e-3 per-row relative
+tolerance, from ragged tiny cases up to the n=8192, batch-64 workload in the
+exact launch configuration the benchmark times."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from decode_attention_cq_b200 import calibq as cq
+from decode_attention_cq_b200 import synth
+
+from _util import OUT_RTOL, f64, ref_output_rounded, row_rel_err
+
+pytestmark = pytest.mark.gpu
+
+CALIBS = [(False, 1.0, 1.0), (True, 0.8, 0.9), (True, 1.0, 0.5), (True, 0.5, 1.0)]
+
+
+def _quant(k, v, device):
+    return (cq.cq_quantize_kv(k.to(device), 1, cq.LAYOUT_OCTET_K),
+            cq.cq_quantize_kv(v.to(device), 1, cq.LAYOUT_OCTET_V))
+
+
+def _ref(q, k, v, calib):
+    dt = "f16" if q.dtype == torch.float16 else "f32"
+    return oracle.decode_attention(f64(q), f64(k), f64(v), 1, dt, calib)["out"]
+
+
+def _err(out, ref, dtype):
+    return row_rel_err(out.float().cpu().numpy(), ref_output_rounded(ref, dtype))
+
+
+@pytest.mark.parametrize("n", [1, 7, 8, 9, 255, 256, 1000, 1024, 1025, 2048, 3328, 4097])
+def test_ragged_lengths(cuda_device, n):
+    q, k, v = synth.make_case(2, 8, 2, n, 128, "f16", outliers=4, seed=n)
+    kq, vq = _quant(k, v, cuda_device)
+    for calib in CALIBS[:2]:
+        out = cq.cq_decode_attn(q.to(cuda_device), kq, vq, calib=calib)
+        torch.cuda.synchronize()
+        assert _err(out, _ref(q, k, v, calib), torch.float16) <= OUT_RTOL, calib
+
+
+@pytest.mark.parametrize("calib", CALIBS)
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+def test_calibration_variants_and_dtypes(cuda_device, calib, dtype):
+    q, k, v = synth.make_case(3, 12, 3, 1500, 128, dtype, outliers=4, seed=77)
+    kq, vq = _quant(k, v, cuda_device)
+    out = cq.cq_decode_attn(q.to(cuda_device), kq, vq, calib=calib)
+    torch.cuda.synchronize()
+    assert _err(out, _ref(q, k, v, calib), q.dtype) <= OUT_RTOL
+
+
+@pytest.mark.parametrize("n", [8192, 16384, 32768])
+def test_long_rows_use_larger_clusters(cuda_device, n):
+    q, k, v = synth.make_case(1, 4, 1, n, 128, "f16", outliers=4, seed=n + 1)
+    kq, vq = _quant(k, v, cuda_device)
+    out = cq.cq_decode_attn(q.to(cuda_device), kq, vq, calib=CALIBS[1])
+    torch.cuda.synchronize()
+    assert _err(out, _ref(q, k, v, CALIBS[1]), torch.float16) <= OUT_RTOL
+
+
+def test_degenerate_inputs(cuda_device):
+    # zero query: all logits equal -> uniform weights (mean of dequantized V)
+    q, k, v = synth.make_case(1, 4, 1, 600, 128, "f16", seed=5)
+    q.zero_()
+    kq, vq = _quant(k, v, cuda_device)
+    out = cq.cq_decode_attn(q.to(cuda_device), kq, vq, calib=CALIBS[1])
+    torch.cuda.synchronize()
+    assert _err(out, _ref(q, k, v, CALIBS[1]), torch.float16) <= OUT_RTOL
+    # constant K and V channels (beta == alpha), single token
+    k2 = torch.full((1, 1, 40, 128), 1.5, dtype=torch.float16)
+    v2 = torch.full((1, 1, 40, 128), -0.75, dtype=torch.float16)
+    q2 = torch.randn(1, 4, 128).half()
+    kq2, vq2 = _quant(k2, v2, cuda_device)
+    out2 = cq.cq_decode_attn(q2.to(cuda_device), kq2, vq2, calib=CALIBS[1]).cpu()
+    assert torch.all(out2 == -0.75)
+    q3, k3, v3 = synth.make_case(2, 8, 2, 1, 128, "f16", seed=6)
+    kq3, vq3 = _quant(k3, v3, cuda_device)
+    out3 = cq.cq_decode_attn(q3.to(cuda_device), kq3, vq3, calib=CALIBS[1]).cpu()
+    assert torch.equal(out3, v3[:, :, 0, :].repeat_interleave(4, dim=1))
+
+
+def test_matches_canonical_path(cuda_device):
+    """The tensor-core path and the CUDA-core path agree on the same cache."""
+    q, k, v = synth.make_case(4, 16, 4, 2000, 128, "f16", outliers=4, seed=8)
+    qd = q.to(cuda_device)
+    kq, vq = _quant(k, v, cuda_device)
+    kc = cq.cq_quantize_kv(k.to(cuda_device), 1, cq.LAYOUT_CANONICAL)
+    vc = cq.cq_quantize_kv(v.to(cuda_device), 1, cq.LAYOUT_CANONICAL)
+    o1 = cq.cq_decode_attn(qd, kq, vq, calib=CALIBS[1]).float().cpu().numpy()
+    o2 = cq.cq_decode_attn(qd, kc, vc, calib=CALIBS[1]).float().cpu().numpy()
+    assert row_rel_err(o1, o2) <= OUT_RTOL
+
+
+def test_repeated_calls_are_deterministic(cuda_device):
+    q, k, v = synth.make_case(2, 8, 2, 3000, 128, "f16", seed=9)
+    kq, vq = _quant(k, v, cuda_device)
+    qd = q.to(cuda_device)
+    o1 = cq.cq_decode_attn(qd, kq, vq, calib=CALIBS[1]).clone()
+    for _ in range(3):
+        o2 = cq.cq_decode_attn(qd, kq, vq, calib=CALIBS[1])
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+
+
+def test_internvl_n3328_batch16_full(cuda_device):
+    """InternVL-2.5-8B layer shape at n=3328, batch 16: every output row."""
+    w = synth.WORKLOADS["internvl8b_n3328_b16"]
+    q, k, v = synth.make_workload(w)
+    kq, vq = _quant(k, v, cuda_device)
+    out = cq.cq_decode_attn(q.to(cuda_device), kq, vq, calib=CALIBS[1])
+    torch.cuda.synchronize()
+    assert _err(out, _ref(q, k, v, CALIBS[1]), torch.float16) <= OUT_RTOL
+
+
+def test_internvl_n8192_batch64_sampled(cuda_device):
+    """The benchmarked workload (n=8192, batch 64, 32/8 heads) in the benchmark's
+    launch configuration; sequences 0, 31 and 63 recomputed by the oracle, and
+    every row checked for the softmax's convex-hull property."""
+    w = synth.WORKLOADS["internvl8b_n8192_b64"]
+    q, k, v = synth.make_workload(w, device=cuda_device)
+    kq, vq = _quant(k, v, cuda_device)
+    out = cq.cq_decode_attn(q, kq, vq, calib=CALIBS[1])
+    torch.cuda.synchronize()
+    for b in (0, 31, 63):
+        ref = _ref(q[b:b + 1].cpu(), k[b:b + 1].cpu(), v[b:b + 1].cpu(), CALIBS[1])
+        assert _err(out[b:b + 1], ref, torch.float16) <= OUT_RTOL, b
+    # every row: o lies within [alpha_V, alpha_V + s_V] per channel (1-bit)
+    a = vq.alpha.float().repeat_interleave(4, dim=1)
+    s = vq.scale.float().repeat_interleave(4, dim=1)
+    o = out.float()
+    tol = 1e-3 * (a.abs() + s.abs())
+    assert torch.all(o >= a - tol) and torch.all(o <= a + s + tol)
+    assert torch.isfinite(o).all()

@@ -1,0 +1,114 @@
+"""GPU parity of cq_quantize_kv and cq_dequant against the fp64 oracle.
+
+Codes, packed bytes (padding included), stored alpha and step must match the
+oracle bit for bit; dequantized values must equal the oracle's float64
+dequantization rounded once to the storage dtype.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from decode_attention_cq_b200 import calibq as cq
+from decode_attention_cq_b200 import synth
+
+from _util import f64, oracle_quantize
+
+pytestmark = pytest.mark.gpu
+
+LAYOUTS = {
+    "canonical": cq.LAYOUT_CANONICAL,
+    "octet_k": cq.LAYOUT_OCTET_K,
+    "octet_v": cq.LAYOUT_OCTET_V,
+}
+
+
+def _cache(B, H, n, dtype, seed, outliers=2):
+    g = torch.Generator().manual_seed(seed)
+    return synth.make_cache(B, H, n, 128, dtype, outliers, g, "cpu")
+
+
+def _check_quantized(x_cpu, qc, bits, layout):
+    ref = oracle_quantize(x_cpu, bits)
+    B, H, n, d = x_cpu.shape
+    alpha = qc.alpha.cpu().numpy()
+    scale = qc.scale.cpu().numpy()
+    assert np.array_equal(alpha.view(np.uint8), ref["alpha"].view(np.uint8)), "alpha differs"
+    assert np.array_equal(scale.view(np.uint8), ref["scale"].view(np.uint8)), "scale differs"
+    packed = qc.codes.cpu().numpy()
+    want = oracle.pack_codes(ref["codes"], layout, bits)
+    assert packed.shape == want.shape
+    if not np.array_equal(packed, want):
+        got = oracle.unpack_codes(packed, layout, n, d, bits)
+        bad = np.argwhere(got != ref["codes"])
+        raise AssertionError(f"{len(bad)} codes differ, first at {bad[:5].tolist()}")
+    return ref
+
+
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
+@pytest.mark.parametrize("n", [1, 7, 300, 1500])
+def test_canonical_codes_bit_exact(cuda_device, dtype, bits, n):
+    x = _cache(2, 3, n, dtype, seed=bits * 100 + n)
+    qc = cq.cq_quantize_kv(x.to(cuda_device), bits, cq.LAYOUT_CANONICAL)
+    torch.cuda.synchronize()
+    _check_quantized(x, qc, bits, cq.LAYOUT_CANONICAL)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+@pytest.mark.parametrize("layout", ["octet_k", "octet_v"])
+@pytest.mark.parametrize("n", [1, 8, 9, 255, 256, 257, 1024, 2049, 3328])
+def test_octet_codes_bit_exact(cuda_device, dtype, layout, n):
+    x = _cache(2, 2, n, dtype, seed=n + 7)
+    qc = cq.cq_quantize_kv(x.to(cuda_device), 1, LAYOUTS[layout])
+    torch.cuda.synchronize()
+    _check_quantized(x, qc, 1, LAYOUTS[layout])
+
+
+def test_exact_ties_and_constant_channels(cuda_device):
+    """Inputs that sit exactly on rounding ties and channels with beta == alpha."""
+    n = 64
+    x = torch.zeros(1, 2, n, 128, dtype=torch.float16)
+    # channel c: values 0 .. 63 * step so (x - alpha) * L / range hits exact halves often
+    for c in range(128):
+        x[0, 0, :, c] = torch.arange(n, dtype=torch.float32) * (0.25 + (c % 5)) - (c % 7)
+    x[0, 1] = 3.5  # every channel constant
+    for bits in (1, 2, 4, 8):
+        for layout in (cq.LAYOUT_CANONICAL,) + ((cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V) if bits == 1 else ()):
+            qc = cq.cq_quantize_kv(x.to(cuda_device), bits, layout)
+            torch.cuda.synchronize()
+            ref = _check_quantized(x, qc, bits, layout)
+            assert np.all(ref["codes"][0, 1] == 0)
+
+
+@pytest.mark.parametrize("layout", ["canonical", "octet_k", "octet_v"])
+def test_dequant_matches_oracle(cuda_device, layout):
+    bits_list = [1, 2, 4, 8] if layout == "canonical" else [1]
+    for dtype in ("f16", "f32"):
+        for bits in bits_list:
+            x = _cache(1, 2, 333, dtype, seed=bits + 3)
+            qc = cq.cq_quantize_kv(x.to(cuda_device), bits, LAYOUTS[layout])
+            got = cq.cq_dequant(qc).cpu()
+            ref = oracle_quantize(x, bits)
+            xh = oracle.dequantize(ref["codes"], ref["alpha"], ref["scale"])
+            want = xh.astype(np.float16 if dtype == "f16" else np.float32)
+            assert np.array_equal(got.numpy().view(np.uint8), want.view(np.uint8))
+
+
+def test_full_size_sampled_rows(cuda_device):
+    """The n=8192, batch-64 workload quantized whole on the GPU; sampled
+    (batch, kv-head) rows checked bit-exactly against the oracle."""
+    w = synth.WORKLOADS["internvl8b_n8192_b64"]
+    q, k, v = synth.make_workload(w, device=cuda_device)
+    for x, layout in ((k, cq.LAYOUT_OCTET_K), (v, cq.LAYOUT_OCTET_V)):
+        qc = cq.cq_quantize_kv(x, 1, layout)
+        torch.cuda.synchronize()
+        for (b, h) in ((0, 0), (17, 3), (63, 7)):
+            xr = x[b:b + 1, h:h + 1].cpu()
+            sub = cq.QuantizedCache(qc.codes[b:b + 1, h:h + 1].contiguous(),
+                                    qc.alpha[b:b + 1, h:h + 1].contiguous(),
+                                    qc.scale[b:b + 1, h:h + 1].contiguous(), layout, 1, w.n)
+            _check_quantized(xr, sub, 1, layout)
+    del q, k, v
+    torch.cuda.empty_cache()
