@@ -28,6 +28,7 @@ ENTRY_POINTS = (
     "cq_codes_bytes",
     "cq_quantize_kv_workspace_size",
     "cq_quantize_kv",
+    "cq_quantize_kv_noalloc",
     "cq_decode_attn_workspace_size",
     "cq_decode_attn",
     "cq_dequant",
@@ -51,6 +52,7 @@ _SIGS = {
     "cq_codes_bytes": ([_I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "cq_quantize_kv_workspace_size": ([_I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "cq_quantize_kv": ([_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P], _I),
+    "cq_quantize_kv_noalloc": ([_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P], _I),
     "cq_decode_attn_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "cq_decode_attn": ([_P, _I, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F,
                         cq_calib, _P, _P, _SZ, _P], _I),
@@ -154,6 +156,24 @@ def cq_quantize_kv(x: torch.Tensor, bits: int, layout: int = LAYOUT_CANONICAL, *
     _check(load().cq_quantize_kv(_ptr(x), _dt(x), B, H, n, d, bits, layout, _ptr(out.codes),
                                  _ptr(out.alpha), _ptr(out.scale), _ptr(workspace),
                                  workspace.numel(), _stream(stream)), "cq_quantize_kv")
+    return out
+
+
+def cq_quantize_kv_noalloc(x: torch.Tensor, bits: int, layout: int = LAYOUT_CANONICAL, *,
+                           out: QuantizedCache | None = None, stream=None) -> QuantizedCache:
+    """cq_quantize_kv with the library's fixed scratch instead of a workspace
+    (for callers that cannot allocate device memory; see include/calibq.h)."""
+    B, H, n, d = x.shape
+    if out is None:
+        nbytes = cq_codes_bytes(layout, B, H, n, d, bits)
+        out = QuantizedCache(
+            codes=torch.empty(B, H, nbytes // (B * H), dtype=torch.uint8, device=x.device),
+            alpha=torch.empty(B, H, d, dtype=x.dtype, device=x.device),
+            scale=torch.empty(B, H, d, dtype=x.dtype, device=x.device),
+            layout=layout, bits=bits, n=n)
+    _check(load().cq_quantize_kv_noalloc(_ptr(x), _dt(x), B, H, n, d, bits, layout, _ptr(out.codes),
+                                         _ptr(out.alpha), _ptr(out.scale), _stream(stream)),
+           "cq_quantize_kv_noalloc")
     return out
 
 

@@ -122,6 +122,25 @@ cq_status cq_quantize_kv(const void* x, cq_dtype dt, int B, int H, int n, int d,
                                          workspace, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+cq_status cq_quantize_kv_noalloc(const void* x, cq_dtype dt, int B, int H, int n, int d, int bits,
+                                 cq_layout layout, uint8_t* codes, void* alpha, void* scale,
+                                 cq_stream_t stream) {
+  if (!valid_dtype(dt)) return CQ_ERR_INVALID_ARG;
+  CQ_TRY(check_shape(B, H, n, d, bits));
+  size_t rb = 0;
+  CQ_TRY(row_bytes(layout, n, bits, &rb));
+  CQ_TRY(check_ptr(x));
+  CQ_TRY(check_ptr(codes));
+  CQ_TRY(check_ptr(alpha));
+  CQ_TRY(check_ptr(scale));
+  if (cq::quantize_workspace_bytes(B * H, n) > cq::quantize_static_scratch_bytes())
+    return CQ_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  if (cq::quantize_static_scratch(&scratch) != cudaSuccess) return CQ_ERR_CUDA;
+  return cuda_status(cq::launch_quantize(x, dt, B * H, n, bits, layout, codes, alpha, scale,
+                                         scratch, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 cq_status cq_decode_attn_workspace_size(cq_layout k_layout, cq_layout v_layout, int B, int Hq,
                                         int Hkv, int n, int d, int bits, size_t* bytes) {
   if (bytes == nullptr) return CQ_ERR_INVALID_ARG;

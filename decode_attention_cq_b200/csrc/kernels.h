@@ -17,6 +17,9 @@ size_t quantize_workspace_bytes(int rows, int n);
 cudaError_t launch_quantize(const void* x, cq_dtype dt, int rows, int n, int bits, cq_layout layout,
                             uint8_t* codes, void* alpha, void* scale, void* workspace,
                             cudaStream_t stream);
+// Device address (current device) and size of the library's fixed quantize scratch.
+size_t quantize_static_scratch_bytes();
+cudaError_t quantize_static_scratch(void** ptr);
 
 // ---- dequant.cu
 cudaError_t launch_dequant(const uint8_t* codes, const void* alpha, const void* scale, cq_dtype dt,

@@ -259,3 +259,42 @@ size_t quantize_workspace_bytes(int rows, int n) {
 }
 
 }  // namespace cq
+
+// ---------------------------------------------------------------------------
+// Fixed scratch for cq_quantize_kv_noalloc: the per-split channel min/max
+// partials live in a file-scope device array instead of a caller workspace.
+// Every GPU that loads the library holds it until the process exits. Host
+// code must not hand the symbol itself to a kernel (it is a host-side stand-in
+// for the device array), so its device address is looked up once per device.
+#include <mutex>
+
+namespace cq {
+
+namespace {
+constexpr size_t kStaticScratchBytes = 4u << 20;  // 4 MiB = 4096 (row, split) partials
+static __device__ __align__(256) unsigned char g_quantize_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 256;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+}  // namespace
+
+size_t quantize_static_scratch_bytes() { return kStaticScratchBytes; }
+
+cudaError_t quantize_static_scratch(void** ptr) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_quantize_scratch);  // with `dev` current
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *ptr = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace cq

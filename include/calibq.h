@@ -134,6 +134,37 @@ cq_status cq_quantize_kv(const void* x, cq_dtype dt, int B, int H, int n, int d,
                          void* workspace, size_t ws_bytes, cq_stream_t stream);
 
 /*
+ * cq_quantize_kv without a caller workspace. (Not part of the method: the
+ * article has no counterpart; this is a deployment convenience.)
+ *
+ * Some embedders cannot give the library scratch device memory: a serving
+ * runtime that has already reserved all of HBM for its own KV-cache pool (a
+ * cudaMalloc there fails or fragments the pool), or a caller on a
+ * latency-critical path where cudaMalloc/cudaFree would implicitly
+ * synchronize the device. This entry point takes the same arguments as
+ * cq_quantize_kv minus the workspace, allocates nothing (no cudaMalloc, no
+ * cudaFree, no allocating library routine) and keeps its scratch -- the
+ * per-split channel minima and maxima -- in a fixed 4 MiB array compiled into
+ * the library, which every GPU that loads the library holds until the
+ * process exits.
+ *
+ *  - Limit: requests whose scratch (cq_quantize_kv_workspace_size) exceeds
+ *    4 MiB return CQ_ERR_UNSUPPORTED and launch nothing.
+ *  - The first call on each device looks up that device's address of the
+ *    array (with the device current); make that first call before any stream
+ *    capture.
+ *  - Every call, on any stream, shares the one array: calls whose kernels
+ *    overlap on the GPU race with each other. Serialize them (one stream, or
+ *    events). The array keeps the previous call's contents; nothing in it has
+ *    to start at zero because every call overwrites what it reads.
+ *  - Unlike the rest of the library this entry point has global state (the
+ *    array and the per-device address cache, guarded by a mutex).
+ */
+cq_status cq_quantize_kv_noalloc(const void* x, cq_dtype dt, int B, int H, int n, int d, int bits,
+                                 cq_layout layout, uint8_t* codes, void* alpha, void* scale,
+                                 cq_stream_t stream);
+
+/*
  * Workspace needed by cq_decode_attn for this layout pair (0 for the octet
  * layouts, which keep every intermediate on chip).
  */
