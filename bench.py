@@ -174,17 +174,25 @@ def run_ours(args, world, rank, local):
     vq = cq.cq_quantize_kv(v, bits, layouts[1], workspace=ws)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
+    def fill():
+        cq.cq_quantize_kv(k, bits, layouts[0], out=kq, workspace=ws)
+        cq.cq_quantize_kv(v, bits, layouts[1], out=vq, workspace=ws)
+
+    fill_graph = torch.cuda.CUDAGraph()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(fill_graph, capture_error_mode="relaxed"):
+        fill()
     fill_ms = []
-    for it in range(3):
+    for it in range(4):
         flush.fill_(it)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        cq.cq_quantize_kv(k, bits, layouts[0], out=kq, workspace=ws)
-        cq.cq_quantize_kv(v, bits, layouts[1], out=vq, workspace=ws)
+        fill_graph.replay()
         e1.record(stream)
         e1.synchronize()
-        fill_ms.append(e0.elapsed_time(e1))
-    del k, v
+        if it:
+            fill_ms.append(e0.elapsed_time(e1))
+    del fill_graph, k, v
     torch.cuda.empty_cache()
 
     out = torch.empty_like(q)
@@ -200,6 +208,34 @@ def run_ours(args, world, rank, local):
         step()
     torch.cuda.synchronize()
 
+    # Host cost of one API call (validation + launch), measured while the GPU
+    # is kept busy so that the host never waits for it.
+    busy = torch.empty(1 << 30, dtype=torch.uint8, device=device)
+    busy.fill_(1)
+    h0 = time.perf_counter()
+    for _ in range(20):
+        step()
+    host_us = (time.perf_counter() - h0) / 20 * 1e6
+    del busy
+    torch.cuda.synchronize()
+
+    # The decode step is replayed from a CUDA graph so that the device time of
+    # a step does not include host launch overhead (reported above).
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        step()
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+        step()
+    torch.cuda.synchronize()
+    for it in range(3):
+        flush.fill_(it)
+        graph.replay()
+    torch.cuda.synchronize()
+
     # ---- timed region: K steps, L2 flushed between steps (outside the events)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -210,7 +246,7 @@ def run_ours(args, world, rank, local):
         for it in range(args.steps):
             flush.fill_((it * 7) & 255)
             starts[it].record(stream)
-            step()
+            graph.replay()
             ends[it].record(stream)
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall0
@@ -275,6 +311,8 @@ def run_ours(args, world, rank, local):
                 "h2d_bytes_per_step": q.numel() * q.element_size(),
                 "d2h_bytes_per_step": out.numel() * out.element_size()},
         "gpu_launches": launches_per_step * args.steps,
+        "host_overhead_us_per_call": host_us,
+        "step_timing": "CUDA events around a CUDA-graph replay of one cq_decode_attn call",
         "clocks": clocks.summary(),
         "wall_s_timed_region": t_wall,
     }
@@ -302,7 +340,11 @@ def run_oracle_sample(w, rows: int, seed: int):
 
 
 def cpu_baseline(w):
-    secs, rows = run_oracle_sample(w, rows=2, seed=99)
+    secs, rows = 0.0, 0
+    while secs < 10.0 and rows < 400:  # about ten seconds of CPU work
+        s, r = run_oracle_sample(w, rows=8, seed=99 + rows)
+        secs += s
+        rows += r
     seqs = rows / w.hkv  # a sequence has Hkv (batch, kv-head) rows
     return {"value": seqs / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{rows} (sequence, kv-head) rows of {args_global.workload} "

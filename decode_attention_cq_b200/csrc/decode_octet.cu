@@ -37,15 +37,18 @@ constexpr int kThreads = 128;
 constexpr int kG = 4;             // query heads per kv-head
 constexpr int kKTile = 1024;      // tokens per K-side tile (128 octets)
 constexpr int kVTile = 256;       // tokens per V-side tile (32 octets)
-constexpr int kMaxSlice = 4096;   // tokens per CTA (logits kept in shared memory)
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColA = 0;     // K: 4 bits x 4 chunks x 8 cols; V: 2 buffers x 8 bits x 8 cols
-constexpr uint32_t kColDK = 128;  // K accumulators: 4 bits x 16 cols
-constexpr uint32_t kColDV = 192;  // V accumulator: 16 cols
+constexpr int kPrefSlice = 2048;  // preferred tokens per CTA (logits kept in shared memory)
+constexpr int kMaxSlice = 8192;   // largest slice: n <= 65536 with 8-CTA clusters
+constexpr int kCtasPerSm = 4;     // 4 x 128 TMEM columns, <= 128 registers per thread
+constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kColA = 0;     // K: 2 buffers x 4 chunks x 8 cols; V: 8 bits x 8 cols
+constexpr uint32_t kColDK = 64;   // K accumulators: 2 buffers x 16 cols
+constexpr uint32_t kColDV = 96;   // V accumulator: 16 cols
 constexpr uint32_t kSpin = 1u << 22;
-constexpr size_t kMinSmem = 80 * 1024;  // keeps at most two CTAs (2 x 256 TMEM columns) per SM
+constexpr size_t kMinSmem = 48 * 1024;  // keeps at most four CTAs (4 x 128 TMEM columns) per SM
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kWMax = (1 << 21) - 1;  // 22-bit signed fixed point for the K-side weights
+constexpr int kVPrefetch = 3;     // V tiles in flight per thread
 
 struct Smem {
   uint8_t bk[4][512];        // K-side B: 32 channels x 16 (head, limb) bytes per chunk, MN-major
@@ -58,7 +61,7 @@ struct Smem {
   float kscale[kG];          // fixed-point step of w_h
   float alog2[kG];           // calibration slope * log2(e)
   float ref[kG];             // largest calibrated logit * log2(e)
-  uint64_t mbar_k;
+  uint64_t mbar_k[2];
   uint64_t mbar_v[2];
   uint32_t tmem_base;
   int err;
@@ -72,6 +75,13 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
+}
+
+// 2^x with the hardware approximation (relative error about 2^-22).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ float warp_min(float v) {
@@ -90,8 +100,13 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// 32 bytes of one V-side lane (channel t of a 256-token tile).
+struct VWords {
+  uint4 lo, hi;
+};
+
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_decode_octet(DecodeArgs a, int cl, int slice_tokens) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>(smem_raw);
@@ -107,6 +122,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kt0 = (int)((rank * nk) / cl), kt1 = (int)(((rank + 1) * nk) / cl);
   const int t0 = kt0 * kKTile, t1 = min(n, kt1 * kKTile);
   const int vt0 = t0 / kVTile, vt1 = (t1 + kVTile - 1) / kVTile;
+  const uint8_t* kc = a.k_codes + (size_t)row * octets * kD;
+  const uint8_t* vc = a.v_codes + (size_t)row * ((n + kVTile - 1) / kVTile) * 4096;
+
+  // The first K tile's codes are requested before anything else so that their
+  // latency overlaps the setup below.
+  uint32_t w32[32];
+  auto load_k_tile = [&](int kt) {
+    const int oct = kt * (kKTile / 8) + t;
+    if (oct < octets) {
+      const uint4* src = reinterpret_cast<const uint4*>(kc + (size_t)oct * kD);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 u = ldg_stream(src + i);
+        w32[4 * i] = u.x;
+        w32[4 * i + 1] = u.y;
+        w32[4 * i + 2] = u.z;
+        w32[4 * i + 3] = u.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) w32[i] = 0;
+    }
+  };
+  if (kt0 < kt1) load_k_tile(kt0);
 
   // ---------------------------------------------------------------- setup
   if (warp == 0) {
@@ -114,7 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tmem_relinquish();
   }
   if (t == 0) {
-    tc::mbar_init(&S.mbar_k, 1);
+    tc::mbar_init(&S.mbar_k[0], 1);
+    tc::mbar_init(&S.mbar_k[1], 1);
     tc::mbar_init(&S.mbar_v[0], 1);
     tc::mbar_init(&S.mbar_v[1], 1);
     tc::fence_mbar_init();
@@ -167,89 +207,81 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
 
   // --------------------------------------------------------------- K side
+  // One step per (tile, bit position k): store the masked codes of bit k into
+  // A[s&1], issue its four chunk MMAs into D[s&1], then finish the previous
+  // step (wait for its MMAs, read D, write logits) while these run.
+  // Logits are kept as scores[h][k][octet] (octet relative to the slice).
   constexpr uint32_t kIdescK = tc::idesc_i8(true, 16);
-  const uint8_t* kc = a.k_codes + (size_t)row * octets * kD;
+  const int slice_oct = slice_tokens / 8;
+  float kscale[kG], c0[kG];
+#pragma unroll
+  for (int h = 0; h < kG; ++h) {
+    kscale[h] = S.kscale[h];
+    c0[h] = S.c0[h];
+  }
   float mn[kG], mx[kG];
 #pragma unroll
   for (int h = 0; h < kG; ++h) {
     mn[h] = FLT_MAX;
     mx[h] = -FLT_MAX;
   }
-  uint32_t phase_k = 0;
-  for (int kt = kt0; kt < kt1; ++kt) {
-    const int oct = kt * (kKTile / 8) + t;
-    uint32_t w32[32];
-    if (oct < octets) {
-      const uint4* src = reinterpret_cast<const uint4*>(kc + (size_t)oct * kD);
+  uint32_t ph_k0 = 0u, ph_k1 = 0u;
+  auto wait_k = [&](int which) {
+    uint32_t& ph = which ? ph_k1 : ph_k0;
+    if (S.err == 0 && !tc::mbar_wait(&S.mbar_k[which], ph, kSpin)) S.err = 1;
+    ph ^= 1u;
+  };
+  // logits of step `sp` (tile kt0 + sp/8, bit sp%8) from D[sp&1]
+  auto finish_k = [&](int sp) {
+    const int buf = sp & 1, k = sp & 7, kt = kt0 + (sp >> 3);
+    wait_k(buf);
+    tc::fence_after_sync();
+    uint32_t dv[16];
+    tc::ld_x16(tbase + lane_off + kColDK + buf * 16, dv);
+    tc::wait_ld();
+    const bool valid = kt * kKTile + 8 * t + k < n;
+    const float pow2 = __int_as_float((127 - k) << 23);  // 2^-k
+    const int o = (kt - kt0) * (kKTile / 8) + t;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint4 u = ldg_stream(src + i);
-        w32[4 * i] = u.x;
-        w32[4 * i + 1] = u.y;
-        w32[4 * i + 2] = u.z;
-        w32[4 * i + 3] = u.w;
+    for (int h = 0; h < kG; ++h) {
+      const float v = fmaf(16384.f, (float)(int)dv[4 * h + 2],
+                           fmaf(128.f, (float)(int)dv[4 * h + 1], (float)(int)dv[4 * h]));
+      const float x = fmaf(v, kscale[h] * pow2, c0[h]);
+      if (valid) {
+        mn[h] = fminf(mn[h], x);
+        mx[h] = fmaxf(mx[h], x);
       }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) w32[i] = 0;
+      scores[((size_t)h * 8 + k) * slice_oct + o] = x;
     }
-#pragma unroll 1
-    for (int r = 0; r < 2; ++r) {
+    tc::fence_before_sync();
+  };
+  const int steps = (kt1 - kt0) * 8;
+  for (int sp = 0; sp < steps; ++sp) {
+    const int buf = sp & 1, k = sp & 7;
+    const uint32_t m = 0x01010101u << k;
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint32_t m = 0x01010101u << (4 * r + kk);
-        uint32_t v[32];
+    for (int c = 0; c < 4; ++c) {
+      uint32_t v[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = w32[i] & m;
-        tc::st_x32(tbase + lane_off + kColA + kk * 32, v);
-      }
-      tc::wait_st();
-      tc::fence_before_sync();
-      __syncthreads();
-      tc::fence_after_sync();
-      const bool live = S.err == 0;
-      if (t == 0 && live) {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            tc::mma_i8_ts(tbase + kColDK + kk * 16, tbase + kColA + kk * 32 + c * 8,
-                          tc::smem_desc(S.bk[c], 128, 512), kIdescK, c > 0 ? 1u : 0u);
-        tc::mma_commit(&S.mbar_k);
-      }
-      if (live && !tc::mbar_wait(&S.mbar_k, phase_k, kSpin)) S.err = 1;
-      phase_k ^= 1;
-      tc::fence_after_sync();
-      uint32_t dv[4][16];
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) tc::ld_x16(tbase + lane_off + kColDK + kk * 16, dv[kk]);
-      tc::wait_ld();
-      float xs[kG][4];
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const int k = 4 * r + kk;
-        const bool valid = kt * kKTile + 8 * t + k < n;
-        const float pow2 = __int_as_float((127 - k) << 23);  // 2^-k
-#pragma unroll
-        for (int h = 0; h < kG; ++h) {
-          const int d0 = (int)dv[kk][4 * h], d1 = (int)dv[kk][4 * h + 1], d2 = (int)dv[kk][4 * h + 2];
-          const float v = (float)(d0 + d1 * 128) + 16384.f * (float)d2;
-          const float x = fmaf(v, S.kscale[h] * pow2, S.c0[h]);
-          xs[h][kk] = x;
-          if (valid) {
-            mn[h] = fminf(mn[h], x);
-            mx[h] = fmaxf(mx[h], x);
-          }
-        }
-      }
-      const int u = kt * kKTile - t0 + 8 * t + 4 * r;
-#pragma unroll
-      for (int h = 0; h < kG; ++h)
-        *reinterpret_cast<float4*>(scores + (size_t)h * slice_tokens + u) =
-            make_float4(xs[h][0], xs[h][1], xs[h][2], xs[h][3]);
-      tc::fence_before_sync();
+      for (int i = 0; i < 8; ++i) v[i] = w32[8 * c + i] & m;
+      tc::st_x8(tbase + lane_off + kColA + buf * 32 + c * 8, v);
     }
+    // all bit positions of this tile are in flight: fetch the next tile
+    if (k == 7 && kt0 + (sp >> 3) + 1 < kt1) load_k_tile(kt0 + (sp >> 3) + 1);
+    tc::wait_st();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (t == 0 && S.err == 0) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tc::mma_i8_ts(tbase + kColDK + buf * 16, tbase + kColA + buf * 32 + c * 8,
+                      tc::smem_desc(S.bk[c], 128, 512), kIdescK, c > 0 ? 1u : 0u);
+      tc::mma_commit(&S.mbar_k[buf]);
+    }
+    if (sp > 0) finish_k(sp - 1);
   }
+  if (steps > 0) finish_k(steps - 1);
 
   // -------------------------------------------- score range of the whole row
 #pragma unroll
@@ -260,6 +292,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       S.red[warp][h][1] = M;
     }
   }
+  // V codes of the first tiles are requested before the cluster exchange.
+  VWords ring[kVPrefetch];
+  auto load_v_tile = [&](int vt, VWords& dst) {
+    if (vt < vt1) {
+      const uint4* src = reinterpret_cast<const uint4*>(vc + (size_t)vt * 4096 + t * 32);
+      dst.lo = ldg_stream(src);
+      dst.hi = ldg_stream(src + 1);
+    }
+  };
+#pragma unroll
+  for (int p = 0; p < kVPrefetch; ++p) load_v_tile(vt0 + p, ring[p]);
   __syncthreads();
   if (t < kG) {
     float m = FLT_MAX, M = -FLT_MAX;
@@ -285,47 +328,55 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
 
   // --------------------------------------------------------------- V side
+  // Per tile: softmax weights -> B (double-buffered in shared memory) while
+  // the previous tile's MMAs run; then wait for them, refill the single A
+  // buffer in TMEM and issue this tile's eight MMAs.
   constexpr uint32_t kIdescV = tc::idesc_i8(false, 16);
-  const uint8_t* vc = a.v_codes + (size_t)row * ((n + kVTile - 1) / kVTile) * 4096;
   const int hp = t & 3, grp = t >> 2;
   const float alog2 = S.alog2[hp], ref = S.ref[hp];
   float lsum = 0.f;
-  uint32_t ph_v[2] = {0u, 0u};
+  uint32_t ph_v0 = 0u, ph_v1 = 0u;  // parity of the next completion of mbar_v[0] / mbar_v[1]
+  auto wait_v = [&](int which) {
+    uint32_t& ph = which ? ph_v1 : ph_v0;
+    if (S.err == 0 && !tc::mbar_wait(&S.mbar_v[which], ph, kSpin)) S.err = 1;
+    ph ^= 1u;
+  };
   for (int vt = vt0; vt < vt1; ++vt) {
     const int it = vt - vt0, buf = it & 1;
-    if (it >= 2) {
-      if (S.err == 0 && !tc::mbar_wait(&S.mbar_v[buf], ph_v[buf], kSpin)) S.err = 1;
-      ph_v[buf] ^= 1;
+    // B: softmax weights of tokens 256 vt + 8 grp + k for head hp, scaled by 2^(31-k)
+    // bv[buf] was last read by the MMAs of tile it-2, waited for in iteration it-1
+    const int i0 = vt * kVTile + 8 * grp;
+    const int o = (i0 - t0) >> 3;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      uint32_t pi = 0;
+      if (i0 + k < n) {
+        const float x = scores[((size_t)hp * 8 + k) * slice_oct + o];
+        const float p = ex2_approx(fmaf(x, alog2, (float)(31 - k) - ref));  // p_i * 2^(31-k)
+        pi = __float2uint_rn(p);
+        lsum = fmaf(p, __int_as_float((127 - 31 + k) << 23), lsum);  // sum_i p_i
+      }
+      *reinterpret_cast<uint32_t*>(&S.bv[buf][k][grp * 16 + 4 * hp]) = pi;
+    }
+    tc::fence_proxy_async();
+    if (it >= 1) {  // the single TMEM A buffer was read by the MMAs of tile it-1
+      wait_v(buf ^ 1);
       tc::fence_after_sync();
     }
     // A: channel t's 32 octet bytes of this tile, one bit position per MMA
-    const uint4* src = reinterpret_cast<const uint4*>(vc + (size_t)vt * 4096 + t * 32);
-    const uint4 u0 = ldg_stream(src), u1 = ldg_stream(src + 1);
-    const uint32_t wv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    const VWords cur = ring[0];
+#pragma unroll
+    for (int p = 0; p + 1 < kVPrefetch; ++p) ring[p] = ring[p + 1];
+    load_v_tile(vt + kVPrefetch, ring[kVPrefetch - 1]);
+    const uint32_t wv[8] = {cur.lo.x, cur.lo.y, cur.lo.z, cur.lo.w, cur.hi.x, cur.hi.y, cur.hi.z, cur.hi.w};
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const uint32_t m = 0x01010101u << k;
       uint32_t v8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) v8[i] = wv[i] & m;
-      tc::st_x8(tbase + lane_off + kColA + buf * 64 + k * 8, v8);
+      tc::st_x8(tbase + lane_off + kColA + k * 8, v8);
     }
-    // B: softmax weights of tokens 256 vt + 8 grp + k for head hp, scaled by 2^(31-k)
-    const int i0 = vt * kVTile + 8 * grp;
-    const float4* sp = reinterpret_cast<const float4*>(scores + (size_t)hp * slice_tokens + (i0 - t0));
-    const float4 s0 = sp[0], s1 = sp[1];
-    const float xs[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      uint32_t pi = 0;
-      if (i0 + k < n) {
-        const float e = fmaf(xs[k], alog2, -ref) + (float)(31 - k);
-        pi = __float2uint_rn(exp2f(e));
-        lsum += (float)pi * __int_as_float((127 - 31 + k) << 23);  // * 2^(k-31)
-      }
-      *reinterpret_cast<uint32_t*>(&S.bv[buf][k][grp * 16 + 4 * hp]) = pi;
-    }
-    tc::fence_proxy_async();
     tc::wait_st();
     tc::fence_before_sync();
     __syncthreads();
@@ -333,19 +384,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (t == 0 && S.err == 0) {
 #pragma unroll
       for (int k = 0; k < 8; ++k)
-        tc::mma_i8_ts(tbase + kColDV, tbase + kColA + buf * 64 + k * 8, tc::smem_desc(S.bv[buf][k], 128, 512),
+        tc::mma_i8_ts(tbase + kColDV, tbase + kColA + k * 8, tc::smem_desc(S.bv[buf][k], 128, 512),
                       kIdescV, (it == 0 && k == 0) ? 0u : 1u);
       tc::mma_commit(&S.mbar_v[buf]);
     }
   }
-  {  // drain the (up to two) outstanding commits
-    const int nit = vt1 - vt0;
-    for (int it = max(0, nit - 2); it < nit; ++it) {
-      const int buf = it & 1;
-      if (S.err == 0 && !tc::mbar_wait(&S.mbar_v[buf], ph_v[buf], kSpin)) S.err = 1;
-      ph_v[buf] ^= 1;
-    }
-  }
+  if (vt1 > vt0) wait_v((vt1 - vt0 - 1) & 1);  // the last tile's commit is the only one not waited for
   tc::fence_after_sync();
   uint32_t dv[16];
   tc::ld_x16(tbase + lane_off + kColDV, dv);
@@ -394,19 +438,51 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) tc::tmem_dealloc(tbase, kTmemCols);
 }
 
+// Cluster size: enough CTAs that each keeps at most kPrefSlice tokens (more
+// only when n needs more than 8 CTAs of that size), then the
+// power of two (<= 8, <= number of K tiles) whose wave count best fills the
+// GPU at kCtasPerSm CTAs per SM.
+int pick_cluster(int rows, int nk, int sms) {
+  int cl = 1;
+  while (cl < 8 && cl * kPrefSlice < nk * kKTile) cl *= 2;
+  if (cl * kMaxSlice < nk * kKTile) return -1;
+  int best = cl;
+  double best_eff = -1.0;
+  for (int c = cl; c <= 8 && c <= nk; c *= 2) {
+    const double waves = (double)rows * c / ((double)sms * kCtasPerSm);
+    const double eff = waves / ceil(waves);
+    if (eff > best_eff + 0.02) {
+      best_eff = eff;
+      best = c;
+    }
+  }
+  return best;
+}
+
 template <typename T>
 cudaError_t run(const DecodeArgs& a, cudaStream_t stream) {
+  static int sms = 0;  // SM count of device 0 class parts; only sizes the cluster choice
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+  }
   const int rows = a.B * a.Hkv;
   const int nk = (a.n + kKTile - 1) / kKTile;
-  int cl = 1;
-  while (cl * kMaxSlice < nk * kKTile) cl *= 2;  // at most kMaxSlice tokens per CTA
-  if (cl > 8) return cudaErrorNotSupported;
-  while (cl < 8 && cl * 2 <= nk && rows * cl < 1184) cl *= 2;  // ~4 waves of 2 CTAs per SM
+  const int cl = pick_cluster(rows, nk, sms);
+  if (cl < 0) return cudaErrorNotSupported;
   const int slice_tokens = ((nk + cl - 1) / cl) * kKTile;
   size_t smem = align1k(sizeof(Smem)) + (size_t)kG * slice_tokens * sizeof(float);
   if (smem < kMinSmem) smem = kMinSmem;
-  cudaError_t e = cudaFuncSetAttribute(k_decode_octet<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  static bool attr_set = false;  // benign race: every caller sets the same value
+  if (!attr_set) {
+    const size_t max_smem = align1k(sizeof(Smem)) + (size_t)kG * kMaxSlice * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(k_decode_octet<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(max_smem > kMinSmem ? max_smem : kMinSmem));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(rows * cl), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

@@ -66,3 +66,15 @@ def test_decode_rejections(cuda_device):
     assert e.value.status == cq.CQ_ERR_INVALID_ARG
     torch.cuda.synchronize()
     assert torch.all(out == 7.0)
+
+
+def test_octet_path_length_limit(cuda_device):
+    """n above 65536 is refused by the tensor-core path (its logits live on chip)."""
+    n = 65537
+    x = torch.zeros(1, 1, n, 128, device=cuda_device).half()
+    kq = cq.cq_quantize_kv(x, 1, cq.LAYOUT_OCTET_K)
+    vq = cq.cq_quantize_kv(x, 1, cq.LAYOUT_OCTET_V)
+    q = torch.zeros(1, 4, 128, device=cuda_device).half()
+    with pytest.raises(cq.CalibqError) as e:
+        cq.cq_decode_attn(q, kq, vq)
+    assert e.value.status == cq.CQ_ERR_UNSUPPORTED

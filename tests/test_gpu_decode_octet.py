@@ -52,7 +52,7 @@ def test_calibration_variants_and_dtypes(cuda_device, calib, dtype):
     assert _err(out, _ref(q, k, v, calib), q.dtype) <= OUT_RTOL
 
 
-@pytest.mark.parametrize("n", [8192, 16384, 32768])
+@pytest.mark.parametrize("n", [8192, 16384, 32768, 65536])
 def test_long_rows_use_larger_clusters(cuda_device, n):
     q, k, v = synth.make_case(1, 4, 1, n, 128, "f16", outliers=4, seed=n + 1)
     kq, vq = _quant(k, v, cuda_device)
