@@ -1,5 +1,7 @@
 // The libcalibq C ABI: host-side validation and dispatch (see include/calibq.h).
 #include <math.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include <limits>
 
@@ -35,6 +37,16 @@ cq_status check_ptr(const void* p) {
   if (cudaGetDevice(&dev) != cudaSuccess) return CQ_ERR_CUDA;
   if (attr.type == cudaMemoryTypeDevice && attr.device != dev) return CQ_ERR_INVALID_ARG;
   return CQ_OK;
+}
+
+// CALIBQ_DECODE_KERNEL=tcgen05 routes every octet-layout decode to the tcgen05
+// kernel (otherwise it serves only rows longer than the mma.sync kernel takes).
+bool force_tcgen05() {
+  static const int forced = [] {
+    const char* v = getenv("CALIBQ_DECODE_KERNEL");
+    return (v != nullptr && strcmp(v, "tcgen05") == 0) ? 1 : 0;
+  }();
+  return forced != 0;
 }
 
 #define CQ_TRY(expr)                 \
@@ -206,7 +218,9 @@ cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, con
     CQ_TRY(check_ptr(workspace));
     return cuda_status(cq::launch_decode_generic(a, dt, workspace, s));
   }
-  const cudaError_t e = cq::launch_decode_octet(a, dt, s);
+  const cudaError_t e = (cq::decode_mma_supports(n) && !force_tcgen05())
+                            ? cq::launch_decode_mma(a, dt, s)
+                            : cq::launch_decode_octet(a, dt, s);
   if (e == cudaErrorNotSupported) return CQ_ERR_UNSUPPORTED;
   return cuda_status(e);
 }

@@ -48,4 +48,8 @@ cudaError_t launch_decode_generic(const DecodeArgs& a, cq_dtype dt, void* worksp
 // ---- decode_octet.cu (octet layouts, bits = 1, Hq = 4 Hkv, tensor cores)
 cudaError_t launch_decode_octet(const DecodeArgs& a, cq_dtype dt, cudaStream_t stream);
 
+// ---- decode_mma.cu (octet layouts, bits = 1, Hq = 4 Hkv, n <= 32768, mma.sync)
+bool decode_mma_supports(int n);
+cudaError_t launch_decode_mma(const DecodeArgs& a, cq_dtype dt, cudaStream_t stream);
+
 }  // namespace cq
