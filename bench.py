@@ -38,7 +38,7 @@ METRIC = "1-bit decode-attention tokens/s and achieved HBM GB/s (n=8192), % of r
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 FALLBACK_HBM_GBS = 6650.0
 CALIB = (True, 0.8, 0.9)
-DECODE_KERNEL_SOURCES = {"octet": "decode_attention_cq_b200/csrc/decode_octet.cu",
+DECODE_KERNEL_SOURCES = {"octet": "decode_attention_cq_b200/csrc/decode_mma.cu",
                          "canonical": "decode_attention_cq_b200/csrc/decode_generic.cu"}
 
 
@@ -304,7 +304,7 @@ def run_ours(args, world, rank, local):
                      "frac": achieved / peak, "peak_source": peak_src,
                      "traffic": None if trec is None else trec["dram_bytes_per_launch"],
                      "algorithmic_bytes_per_launch": alg,
-                     "kernel": "cq_decode_attn " + args.path},
+                     "kernel": "k_decode_mma" if args.path == "octet" else "k_scores + k_softmax_v + k_merge"},
         "cache_fill": {"ms": fill_mean, "algorithmic_bytes": fill_alg,
                        "achieved_gbs": fill_alg / (fill_mean * 1e-3) / 1e9},
         "e2e": {"value": total_tokens / (e2e_mean * 1e-3), "unit": "tokens/s",

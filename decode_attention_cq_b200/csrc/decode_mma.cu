@@ -8,21 +8,24 @@
 // sum_i p_i c^V_i / sum_i p_i (Method 2 applied to V).
 //
 // One thread-block cluster per (batch, kv-head) row, one CTA per slice of at
-// most 2048 tokens (4096 for n > 16384). Each CTA
+// most S tokens (S = 2048, or 4096 for n > 16384). Each CTA
 //  1. streams its slice of K and V codes into shared memory with cp.async
 //     (16-byte chunks, XOR-swizzled so that ldmatrix reads are conflict-free);
 //  2. K side: per unit of 16 token octets (128 tokens) a warp loads the A
 //     fragments of all 128 channels with ldmatrix; masking bit k of every byte
 //     gives "code of token 8 r + k times 2^k" for octet row r. B holds the
 //     weights w_h = sigma q_h (.) s_K as a 22-bit fixed-point number split into
-//     three int8 limbs (two N = 8 tiles: heads x limbs);
+//     three int8 limbs (two N = 8 tiles: heads x limbs). The unit's logits
+//     (2 KB) overwrite its codes (2 KB), which the warp holds in registers;
 //  3. exchanges the logit range with the other CTAs of the row (distributed
-//     shared memory), computes the calibration slope and the softmax weights
-//     p_i 2^(31-k) as four uint8 limbs, written straight in A-fragment order;
-//  4. V side: A = weight limbs (16 rows = 4 limbs x 4 heads, K = 32 octets of
-//     one bit position), B = masked codes of 8 channels (ldmatrix); every warp
-//     accumulates sum_i c_ij p_i 2^31 for all 128 channels in 64 registers;
-//  5. sums the warps and the cluster and writes o.
+//     shared memory) and derives the calibration slope;
+//  4. turns logits into softmax weights p_i 2^(31-k) as four uint8 limbs,
+//     written in A-fragment order over the logits;
+//  5. V side: A = weight limbs (16 rows = 4 limbs x 4 heads, K = 32 octets of
+//     one bit position), B = masked codes of 8 channels (ldmatrix); a warp
+//     pair splits the 128 channels, the four pairs split the tiles;
+//  6. sums the warps, scatters the (head, channel) partial sums over the
+//     cluster so that every CTA owns a range of channels, and writes o.
 // Everything stays on chip; one launch per decode step, no workspace.
 #include <float.h>
 
@@ -37,27 +40,29 @@ namespace {
 constexpr int kThreads = 256;  // 8 warps
 constexpr int kWarps = kThreads / 32;
 constexpr int kG = 4;          // query heads per kv-head
-constexpr int kUnit = 128;     // tokens per K-side unit (16 octets)
-constexpr int kVTile = 256;    // tokens per V-side tile (32 octets)
+constexpr int kUnit = 128;     // tokens per K-side unit (16 octets, 2 KB of codes)
+constexpr int kVTile = 256;    // tokens per V-side tile (32 octets, 4 KB of codes)
 constexpr int kMaxCl = 8;
 constexpr int kWMax = (1 << 21) - 1;
+constexpr int kLimbRow = 132;  // bytes per limb row (padding spreads the B-fragment loads over banks)
+constexpr int kRecv = kG * 136;  // >= kG * cl * ceil(kD / cl) for every cl <= 8
+constexpr int kPartStride = kD + 8;  // floats per (warp pair, head) row of the partial sums
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Shared memory, slice of S tokens: K codes S/8 x 128 B | V codes S/256 x 4 KB |
-// logits 32 rows (bit position, head) x (S/8 + 8) floats | fixed part below |
-// rank 0 only: the cluster's partial sums.
 struct Fixed {
-  int wint[kG][kD];             // K-side weights in fixed point
-  float red[kWarps][kG][2];     // per-warp reduction scratch
-  float mM[kMaxCl][kG][2];      // every peer's logit range per head (pushed to all)
-  float part_l[kMaxCl][kG];     // every peer's sum of weights (pushed to rank 0)
-  float lsum[kWarps][kG];       // per-warp sum of weights
+  uint8_t limb[kG * 3][kLimbRow];  // K-side weight limbs: row 3 h + l, byte = channel
+  float red[kWarps][kG][2];        // per-warp reduction scratch
+  float mM[kMaxCl][kG][2];         // every peer's logit range per head (pushed to all)
+  float part_l[kMaxCl][kG];        // every peer's sum of weights (pushed to all)
+  float lsum[kWarps][kG];          // per-warp sum of weights
   float c0[kG], kscale[kG], alog2[kG], ref[kG];
+  float recv[kRecv];               // [src][h][channel - first owned channel], stride ceil(kD / cl)
 };
 
+// Shared memory for a slice of S tokens: K codes / logits / weight fragments
+// (S/8 x 128 B) | V codes / partial sums (S/256 x 4 KB) | fixed part.
 __host__ __device__ constexpr size_t smem_bytes(int slice) {
-  return (size_t)slice / 8 * 128 + (size_t)slice / kVTile * 4096 + (size_t)8 * kG * (slice / 8 + 8) * 4 +
-         sizeof(Fixed);
+  return (size_t)slice / 8 * 128 + (size_t)slice / kVTile * 4096 + sizeof(Fixed);
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
@@ -73,22 +78,30 @@ __device__ __forceinline__ void cp_async_wait() {
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void lds128(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
 }
 
-// D += A (16x32 u8, row) x B (32x8 s8, col)
+// D += A (16x32 u8, row) x B (32x8 s8, col). Register-only: the compiler may
+// interleave independent MMAs.
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-               "{%0,%1,%2,%3};"
-               : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 // D += A (16x32 u8, row) x B (32x8 u8, col)
 __device__ __forceinline__ void mma_u8u8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-               "{%0,%1,%2,%3};"
-               : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -107,20 +120,23 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Slice capacity S (tokens, multiple of 256, >= 1024) and cluster size cl.
-template <typename T>
-__global__ void __launch_bounds__(kThreads, 2) k_decode_mma(DecodeArgs a, int cl, int S) {
+// Position (in floats, within its unit's 2 KB) of the logit of octet o (0..15)
+// of a unit, bit position k, head h. Rows of 16 floats; odd units swap row
+// pairs and heads 2, 3 swap octet halves, so that both the K-side stores and
+// the softmax-side float4 loads are free of bank conflicts.
+__device__ __forceinline__ int logit_pos(int unit, int k, int h, int o) {
+  return (((k * kG + h) ^ (unit & 1)) << 4) + (o ^ ((h >> 1) << 3));
+}
+
+template <typename T, int S>
+__global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1) k_decode_mma(DecodeArgs a, int cl) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // logit rows are S/8 + 8 floats apart: the K-side stores of the four heads of
-  // one octet then hit four different bank groups
-  const int so = S / 8 + 8;
-  uint8_t* sK = smem_raw;                                 // [S/8][128], 16-byte chunks swizzled by octet
-  uint8_t* sV = sK + (size_t)S / 8 * 128;                 // [S/256][128][32], halves swizzled by channel
-  float* sS = reinterpret_cast<float*>(sV + (size_t)S / kVTile * 4096);  // logits [k][h][octet]
-  Fixed& F = *reinterpret_cast<Fixed*>(reinterpret_cast<uint8_t*>(sS) + (size_t)8 * kG * so * 4);
-  float* gather = reinterpret_cast<float*>(&F + 1);       // [cl][kG][kD] partial sums pushed to rank 0
-  uint8_t* sFrag = sK;                                    // weight-limb A fragments (after the K side)
-  float* sPart = sS;                                      // per-warp partial sums (after step 5)
+  uint8_t* sK = smem_raw;                      // [S/8][128] codes, 16-byte chunks swizzled by octet
+  uint8_t* sV = sK + (size_t)S / 8 * 128;      // [S/256][128][32] codes, halves swizzled by channel
+  Fixed& F = *reinterpret_cast<Fixed*>(sV + (size_t)S / kVTile * 4096);
+  float* sL = reinterpret_cast<float*>(sK);    // logits, unit u at floats [512 u, 512 u + 512)
+  uint8_t* sFrag = sK;                         // weight-limb A fragments, tile lt at bytes [4096 lt, ...)
+  float* sPart = reinterpret_cast<float*>(sV);  // per warp-pair partial sums (after the V side)
 
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31, g = lane >> 2, tq = lane & 3;
   const uint32_t rank = tc::cluster_rank();
@@ -131,9 +147,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_mma(DecodeArgs a, int cl
   const int nvt = (n + kVTile - 1) / kVTile;
   const int vt0 = (int)((rank * nvt) / cl), vt1 = (int)(((rank + 1) * nvt) / cl);
   const int t0 = vt0 * kVTile, t1 = min(n, vt1 * kVTile);
-  const int nvtl = vt1 - vt0;                     // V tiles of this CTA
+  const int nvtl = vt1 - vt0;                        // V tiles of this CTA
   const int nunits = (t1 - t0 + kUnit - 1) / kUnit;  // K units of this CTA
-  const uint32_t sK_u = tc::smem_u32(sK), sV_u = tc::smem_u32(sV), sF_u = tc::smem_u32(sFrag);
+  const uint32_t sK_u = tc::smem_u32(sK), sV_u = tc::smem_u32(sV);
 
   // ---- 1. stream this slice's codes into shared memory (K first, then V)
   {
@@ -156,11 +172,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_mma(DecodeArgs a, int cl
   tc::cluster_arrive_relaxed();  // matched by the wait before the first peer store
 
   // ---- 2. post-scaled K weights w_h = sigma q_h (.) s_K in 22-bit fixed point
+  float w[kG];
   if (t < kD) {
     const T* qp = static_cast<const T*>(a.q) + ((size_t)b * a.Hq + (size_t)kG * hkv) * kD;
     const float sk = DT<T>::f(static_cast<const T*>(a.k_scale)[(size_t)row * kD + t]);
     const float ak = DT<T>::f(static_cast<const T*>(a.k_alpha)[(size_t)row * kD + t]);
-    float w[kG];
 #pragma unroll
     for (int h = 0; h < kG; ++h) {
       const float qv = DT<T>::f(qp[h * kD + t]);
@@ -172,49 +188,35 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_mma(DecodeArgs a, int cl
         F.red[warp][h][1] = qa;
       }
     }
-    __syncwarp();
-    // every warp of the first four needs all four warps' maxima: done after the barrier
-#pragma unroll
-    for (int h = 0; h < kG; ++h) F.wint[h][t] = __float_as_int(w[h]);  // raw weight, scaled below
-  }
-  __syncthreads();
-  if (t < kG) {
-    float amax = 0.f, qa = 0.f;
-    for (int q = 0; q < 4; ++q) {
-      amax = fmaxf(amax, F.red[q][t][0]);
-      qa += F.red[q][t][1];
-    }
-    F.c0[t] = a.sigma * qa;
-    F.kscale[t] = amax > 0.f ? amax / (float)kWMax : 0.f;
   }
   __syncthreads();
   if (t < kD) {
 #pragma unroll
     for (int h = 0; h < kG; ++h) {
-      const float inv = F.kscale[h] > 0.f ? 1.f / F.kscale[h] : 0.f;
-      const int wi = __float2int_rn(__int_as_float(F.wint[h][t]) * inv);
-      F.wint[h][t] = max(-kWMax, min(kWMax, wi));
+      const float amax = fmaxf(fmaxf(F.red[0][h][0], F.red[1][h][0]), fmaxf(F.red[2][h][0], F.red[3][h][0]));
+      const float ks = amax > 0.f ? amax / (float)kWMax : 0.f;
+      const float inv = ks > 0.f ? 1.f / ks : 0.f;
+      const int wi = max(-kWMax, min(kWMax, __float2int_rn(w[h] * inv)));
+      F.limb[3 * h + 0][t] = (uint8_t)(wi & 127);
+      F.limb[3 * h + 1][t] = (uint8_t)((wi >> 7) & 127);
+      F.limb[3 * h + 2][t] = (uint8_t)((wi >> 14) & 255);
+      if (t == h) {
+        F.kscale[h] = ks;
+        F.c0[h] = a.sigma * (F.red[0][h][1] + F.red[1][h][1] + F.red[2][h][1] + F.red[3][h][1]);
+      }
     }
   }
   __syncthreads();
-  // B fragments of the K side: bk[c][tile][half], channel 32c + 16 half + 4 tq + i;
-  // tile 0 column g = (head g/2, limb g%2), tile 1 column g = (head g/2, limb 2) for even g.
+  // B fragments of the K side: bk[c][tile][half] holds channels 32c + 16 half + 4 tq + (0..3);
+  // tile 0 column g = (head g/2, limb g%2), tile 1 column g = (head g/2, limb 2) for even g, 0 for odd g.
   uint32_t bk[4][2][2];
 #pragma unroll
   for (int c = 0; c < 4; ++c)
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-      uint32_t r0 = 0, r1 = 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int w = F.wint[g >> 1][32 * c + 16 * half + 4 * tq + i];
-        const uint32_t l01 = (g & 1) ? ((w >> 7) & 127) : (w & 127);
-        const uint32_t l2 = (g & 1) ? 0u : (uint32_t)((w >> 14) & 255);
-        r0 |= l01 << (8 * i);
-        r1 |= l2 << (8 * i);
-      }
-      bk[c][0][half] = r0;
-      bk[c][1][half] = r1;
+      const int j = 32 * c + 16 * half + 4 * tq;
+      bk[c][0][half] = *reinterpret_cast<const uint32_t*>(&F.limb[3 * (g >> 1) + (g & 1)][j]);
+      bk[c][1][half] = (g & 1) ? 0u : *reinterpret_cast<const uint32_t*>(&F.limb[3 * (g >> 1) + 2][j]);
     }
   const float c0 = F.c0[tq], kscale = F.kscale[tq];
 
@@ -226,59 +228,64 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_mma(DecodeArgs a, int cl
     uint32_t af[4][4];  // A fragments of chunks c = 0..3 (rows = octets 16u + {g, g+8})
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const int m = lane >> 3, lo = 16 * u + 8 * (m & 1) + (lane & 7), c16 = 2 * c + (m >> 1);
-      ldsm_x4(sK_u + lo * 128 + ((c16 ^ (lo & 7)) << 4), af[c]);
+      const int m = lane >> 3, r8 = 8 * (m & 1) + (lane & 7), c16 = 2 * c + (m >> 1);
+      ldsm_x4(sK_u + u * 2048 + r8 * 128 + ((c16 ^ (lane & 7)) << 4), af[c]);
     }
-    float xs[2][8];
+    float* lg = sL + u * 512;  // this unit's logits overwrite its codes (held in af)
+    const int tok = t0 + kUnit * u + 8 * g;  // token of octet row g, bit 0
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t msk = 0x01010101u << k;
-      int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
+    for (int k = 0; k < 8; k += 2) {
+      int d[2][2][4];  // [bit k + kk][tile][reg]
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint32_t am[4] = {af[c][0] & msk, af[c][1] & msk, af[c][2] & msk, af[c][3] & msk};
-        mma_u8s8(d0, am, bk[c][0][0], bk[c][0][1]);
-        mma_u8s8(d1, am, bk[c][1][0], bk[c][1][1]);
-      }
-      // d0 = (row g | g+8, cols 2tq, 2tq+1) = head tq limbs 0, 1; d1 cols 2tq = head tq limb 2
-      const float sc = kscale * __int_as_float((127 - k) << 23);  // step * 2^-k
+      for (int kk = 0; kk < 2; ++kk)
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const float v = fmaf(16384.f, (float)d1[2 * r], fmaf(128.f, (float)d0[2 * r + 1], (float)d0[2 * r]));
-        const float x = fmaf(v, sc, c0);
-        xs[r][k] = x;
-        if (t0 + 8 * (16 * u + g + 8 * r) + k < t1) {
-          mn = fminf(mn, x);
-          mx = fmaxf(mx, x);
+        for (int tl = 0; tl < 2; ++tl) d[kk][tl][0] = d[kk][tl][1] = d[kk][tl][2] = d[kk][tl][3] = 0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint32_t msk = 0x01010101u << (k + kk);
+          const uint32_t am[4] = {af[c][0] & msk, af[c][1] & msk, af[c][2] & msk, af[c][3] & msk};
+          mma_u8s8(d[kk][0], am, bk[c][0][0], bk[c][0][1]);
+          mma_u8s8(d[kk][1], am, bk[c][1][0], bk[c][1][1]);
+        }
+      // d[kk][0] = (row g | g+8, cols 2tq, 2tq+1) = head tq limbs 0, 1; d[kk][1] col 2tq = head tq limb 2
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk) {
+        const float sc = kscale * __int_as_float((127 - k - kk) << 23);  // step * 2^-k
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float v = fmaf(16384.f, (float)d[kk][1][2 * r],
+                               fmaf(128.f, (float)d[kk][0][2 * r + 1], (float)d[kk][0][2 * r]));
+          const float x = fmaf(v, sc, c0);
+          if (tok + 64 * r + k + kk < t1) {
+            mn = fminf(mn, x);
+            mx = fmaxf(mx, x);
+          }
+          lg[logit_pos(u, k + kk, tq, g + 8 * r)] = x;
         }
       }
     }
-    // logits as sS[k][h][octet]
-#pragma unroll
-    for (int r = 0; r < 2; ++r)
-#pragma unroll
-      for (int k = 0; k < 8; ++k) sS[(k * kG + tq) * so + 16 * u + g + 8 * r] = xs[r][k];
   }
 
   // ---- 4. logit range of the whole row (cluster), calibration slope
-  {
-    // lanes with equal tq hold the same head
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 4));
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 8));
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 16));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    if (lane < kG) {
-      F.red[warp][lane][0] = mn;
-      F.red[warp][lane][1] = mx;
-    }
+  // lanes with equal tq hold the same head
+  mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 4));
+  mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 8));
+  mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 16));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+  if (lane < kG) {
+    F.red[warp][lane][0] = mn;
+    F.red[warp][lane][1] = mx;
   }
   __syncthreads();
   tc::cluster_wait();  // every CTA of the cluster is running
   if (t < kG * kMaxCl) {  // thread (h, r): push this CTA's range of head h to peer r
     const int h = t & 3, r = t >> 2;
     float m = FLT_MAX, M = -FLT_MAX;
+#pragma unroll
     for (int q = 0; q < kWarps; ++q) {
       m = fminf(m, F.red[q][h][0]);
       M = fmaxf(M, F.red[q][h][1]);
@@ -302,37 +309,49 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_mma(DecodeArgs a, int cl
   }
   __syncthreads();
 
-  // ---- 5. softmax weights P = p_i 2^(31-k) as four uint8 limbs, stored in the
-  // A-fragment order of the V side (sFrag reuses the K codes' space). Thread
-  // (k = warp, h, grp) takes the tokens 8 (4 grp + j) + k, j = 0..3, of every V
-  // tile; A row m = 4 limb + h, A column = octet within the tile.
+  // ---- 5. softmax weights P = p_i 2^(31-k) as four uint8 limbs in the A-fragment
+  // order of the V side, over the logits. Thread (k = warp, h, grp) takes the
+  // tokens 8 (4 grp + j) + k, j = 0..3, of every V tile; A row m = 4 limb + h,
+  // A column = octet within the tile. A tile's logits are all read (group of
+  // up to 8 tiles, then a barrier) before its fragments are written.
   float lsum = 0.f;
   {
     const int k = warp, h = (lane >> 3) & 3, grp = lane & 7;
     const float alog2 = F.alog2[h], bias = (float)(31 - k) - F.ref[h];
     const float unscale = __int_as_float((127 - 31 + k) << 23);  // 2^(k-31)
-    const float* src = sS + (k * kG + h) * so + 4 * grp;
+    // octets 4 grp .. 4 grp + 3 of tile lt: unit 2 lt + grp / 4, octets 4 (grp % 4) ..
+    const float* src = sL + (grp >> 2) * 512 + logit_pos(grp >> 2, k, h, 4 * (grp & 3));
     // lane 4 h + grp % 4 holds A rows h (limb 0) and h + 8 (limb 2); lane + 16 rows h + 4, h + 12
     uint8_t* dst = sFrag + (size_t)(k * 32 + 4 * h + (grp & 3)) * 16 + (grp >> 2) * 8;
-    for (int lt = 0; lt < nvtl; ++lt) {
-      const float4 x4 = *reinterpret_cast<const float4*>(src + lt * 32);
-      const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
-      const int i0 = t0 + lt * kVTile + 32 * grp + k;  // token of j = 0
-      uint32_t P[4];
+#pragma unroll 1
+    for (int lt0 = 0; lt0 < nvtl; lt0 += 8) {
+      float4 xv[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const bool ok = i0 + 8 * j < t1;
-        const float p = ex2_approx(fmaf(xv[j], alog2, bias));
-        P[j] = ok ? __float2uint_rn(p) : 0u;
-        lsum += ok ? p * unscale : 0.f;
+      for (int i = 0; i < 8; ++i)
+        if (lt0 + i < nvtl) xv[i] = *reinterpret_cast<const float4*>(src + (lt0 + i) * 1024);
+      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int lt = lt0 + i;
+        if (lt >= nvtl) break;
+        const float xs[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+        const int i0 = t0 + lt * kVTile + 32 * grp + k;  // token of j = 0
+        uint32_t P[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const bool ok = i0 + 8 * j < t1;
+          const float p = ex2_approx(fmaf(xs[j], alog2, bias));
+          P[j] = ok ? __float2uint_rn(p) : 0u;
+          lsum += ok ? p * unscale : 0.f;
+        }
+        // word l = byte l of P[0..3]
+        const uint32_t lo01 = __byte_perm(P[0], P[1], 0x5140), hi01 = __byte_perm(P[0], P[1], 0x7362);
+        const uint32_t lo23 = __byte_perm(P[2], P[3], 0x5140), hi23 = __byte_perm(P[2], P[3], 0x7362);
+        const uint32_t w0 = __byte_perm(lo01, lo23, 0x5410), w1 = __byte_perm(lo01, lo23, 0x7632);
+        const uint32_t w2 = __byte_perm(hi01, hi23, 0x5410), w3 = __byte_perm(hi01, hi23, 0x7632);
+        *reinterpret_cast<uint2*>(dst + (size_t)lt * 4096) = make_uint2(w0, w2);
+        *reinterpret_cast<uint2*>(dst + (size_t)lt * 4096 + 256) = make_uint2(w1, w3);
       }
-      // word l = byte l of P[0..3]
-      const uint32_t lo01 = __byte_perm(P[0], P[1], 0x5140), hi01 = __byte_perm(P[0], P[1], 0x7362);
-      const uint32_t lo23 = __byte_perm(P[2], P[3], 0x5140), hi23 = __byte_perm(P[2], P[3], 0x7362);
-      const uint32_t w0 = __byte_perm(lo01, lo23, 0x5410), w1 = __byte_perm(lo01, lo23, 0x7632);
-      const uint32_t w2 = __byte_perm(hi01, hi23, 0x5410), w3 = __byte_perm(hi01, hi23, 0x7632);
-      *reinterpret_cast<uint2*>(dst + (size_t)lt * 4096) = make_uint2(w0, w2);
-      *reinterpret_cast<uint2*>(dst + (size_t)lt * 4096 + 256) = make_uint2(w1, w3);
     }
     // lanes with equal h: xor over grp
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
@@ -343,46 +362,43 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_mma(DecodeArgs a, int cl
   cp_async_wait<0>();  // V codes
   __syncthreads();
 
-  // ---- 6. V side: warp w takes tiles w, w + 8, ...; D rows (limb, head), columns channels
-  int acc[16][4];
+  // ---- 6. V side: warp pair p = warp / 2 takes tiles p, p + 4, ...; warp parity
+  // picks channels 64 hc .. 64 hc + 63. D rows (limb, head), columns channels.
+  const int hc = warp & 1, pair = warp >> 1;
+  int acc[8][4];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0;
-  for (int lt = warp; lt < nvtl; lt += kWarps) {
-    const uint32_t tile_u = sV_u + lt * 4096, frag_u = sF_u + lt * 4096 + lane * 16;
+  for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0;
+  for (int lt = pair; lt < nvtl; lt += kWarps / 2) {
+    const uint32_t tile_u = sV_u + lt * 4096, frag_u = sK_u + lt * 4096 + lane * 16;
+    uint32_t bv[8][2];
 #pragma unroll
-    for (int hc = 0; hc < 2; ++hc) {  // channels 64 hc .. 64 hc + 63
-      uint32_t bv[8][2];
+    for (int p = 0; p < 4; ++p) {
+      const int mat = lane >> 3, half = mat & 1;
+      const int ch = 64 * hc + 16 * p + 8 * (mat >> 1) + (lane & 7);
+      uint32_t r[4];
+      ldsm_x4(tile_u + ch * 32 + ((half ^ ((ch >> 2) & 1)) << 4), r);
+      bv[2 * p][0] = r[0];
+      bv[2 * p][1] = r[1];
+      bv[2 * p + 1][0] = r[2];
+      bv[2 * p + 1][1] = r[3];
+    }
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const int mat = lane >> 3, half = mat & 1;
-        const int ch = 64 * hc + 16 * p + 8 * (mat >> 1) + (lane & 7);
-        uint32_t r[4];
-        ldsm_x4(tile_u + ch * 32 + ((half ^ ((ch >> 2) & 1)) << 4), r);
-        bv[2 * p][0] = r[0];
-        bv[2 * p][1] = r[1];
-        bv[2 * p + 1][0] = r[2];
-        bv[2 * p + 1][1] = r[3];
-      }
+    for (int k = 0; k < 8; ++k) {
+      uint32_t af[4];
+      lds128(frag_u + k * 512, af);
+      const uint32_t msk = 0x01010101u << k;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        uint32_t af[4];
-        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(af[0]), "=r"(af[1]), "=r"(af[2]), "=r"(af[3])
-                     : "r"(frag_u + k * 512));
-        const uint32_t msk = 0x01010101u << k;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) mma_u8u8(acc[8 * hc + j], af, bv[j][0] & msk, bv[j][1] & msk);
-      }
+      for (int j = 0; j < 8; ++j) mma_u8u8(acc[j], af, bv[j][0] & msk, bv[j][1] & msk);
     }
   }
 
-  // ---- 7. combine limbs (lane and lane ^ 16), sum the warps, push to rank 0
-  // lane with g < 4 holds limbs 0 and 2 of head g, lane + 16 limbs 1 and 3
-  constexpr int kPartStride = kD + 8;  // floats per (warp, head) row of sPart
+  // ---- 7. combine limbs (lane and lane ^ 16), sum the warp pairs, scatter to the owners
+  // Lane with g < 4 holds limbs 0 and 2 of head g, lane + 16 limbs 1 and 3.
+  __syncthreads();  // every warp is done with the V codes: the partial sums reuse them
   {
     const float s_lo = (g < 4) ? 0x1p-31f : 0x1p-23f, s_hi = (g < 4) ? 0x1p-15f : 0x1p-7f;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
+    for (int j = 0; j < 8; ++j) {
       float v[2];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -390,70 +406,67 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_mma(DecodeArgs a, int cl
         v[c] += __shfl_xor_sync(0xffffffffu, v[c], 16);
       }
       if (lane < 16)
-        *reinterpret_cast<float2*>(sPart + (warp * kG + g) * kPartStride + 8 * j + 2 * tq) = make_float2(v[0], v[1]);
+        *reinterpret_cast<float2*>(sPart + (pair * kG + g) * kPartStride + 64 * hc + 8 * j + 2 * tq) =
+            make_float2(v[0], v[1]);
     }
   }
   __syncthreads();
-  {
-    float* gather_r = gather + (size_t)rank * kG * kD;
+  // CTA r of the cluster owns channels [r kD / cl, (r + 1) kD / cl); recv rows are ceil(kD / cl) wide
+  const int wrecv = (kD + cl - 1) / cl;
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int idx = 2 * t + e, h = idx >> 7, ch = idx & 127;
-      float s = 0.f;
+  for (int e = 0; e < 2; ++e) {
+    const int idx = 2 * t + e, h = idx >> 7, ch = idx & 127;
+    float s = 0.f;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) s += sPart[(w * kG + h) * kPartStride + ch];
-      tc::st_peer_f32(gather_r + h * kD + ch, 0, s);
-    }
-    if (t < kG) {
+    for (int q = 0; q < kWarps / 2; ++q) s += sPart[(q * kG + h) * kPartStride + ch];
+    int owner = 0;
+    while ((owner + 1) * kD / cl <= ch) ++owner;
+    const int first = owner * kD / cl;
+    tc::st_peer_f32(&F.recv[((int)rank * kG + h) * wrecv + ch - first], (uint32_t)owner, s);
+  }
+  if (t < kG * kMaxCl) {  // thread (h, r): this CTA's sum of weights of head h to peer r
+    const int h = t & 3, r = t >> 2;
+    if (r < cl) {
       float l = 0.f;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) l += F.lsum[w][t];
-      tc::st_peer_f32(&F.part_l[rank][t], 0, l);
+      for (int q = 0; q < kWarps; ++q) l += F.lsum[q][h];
+      tc::st_peer_f32(&F.part_l[rank][h], (uint32_t)r, l);
     }
   }
   tc::cluster_sync();
 
-  // ---- 8. rank 0 merges the cluster: o = alpha_V + s_V (.) sum c p / sum p
-  if (rank == 0) {
-    const int ch = t & 127;
-    const size_t kv = (size_t)row * kD + ch;
-    const float alpha = DT<T>::f(static_cast<const T*>(a.v_alpha)[kv]);
-    const float step = DT<T>::f(static_cast<const T*>(a.v_scale)[kv]);
-    T* out = static_cast<T*>(a.out) + ((size_t)b * a.Hq + (size_t)kG * hkv) * kD;
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int h = 2 * (t >> 7) + e;
+  // ---- 8. every CTA finishes its channels: o = alpha_V + s_V (.) sum c p / sum p
+  {
+    const int first = (int)rank * kD / cl, width = ((int)rank + 1) * kD / cl - first;
+    for (int e = t; e < kG * width; e += kThreads) {
+      const int h = e / width, ch = first + e % width;
       float s = 0.f, l = 0.f;
       for (int r = 0; r < cl; ++r) {
-        s += gather[((size_t)r * kG + h) * kD + ch];
+        s += F.recv[(r * kG + h) * wrecv + ch - first];
         l += F.part_l[r][h];
       }
-      out[h * kD + ch] = DT<T>::from_float(fmaf(step, s / l, alpha));
+      const size_t kv = (size_t)row * kD + ch;
+      const float alpha = DT<T>::f(static_cast<const T*>(a.v_alpha)[kv]);
+      const float step = DT<T>::f(static_cast<const T*>(a.v_scale)[kv]);
+      T* out = static_cast<T*>(a.out) + ((size_t)b * a.Hq + (size_t)kG * hkv + h) * kD;
+      out[ch] = DT<T>::from_float(fmaf(step, s / l, alpha));
     }
   }
 }
 
-template <typename T>
-cudaError_t run(const DecodeArgs& a, cudaStream_t stream) {
-  const int rows = a.B * a.Hkv;
-  const int nvt = (a.n + kVTile - 1) / kVTile;
-  const int S = nvt <= 64 ? 2048 : 4096;  // 2 CTAs per SM up to n = 16384, then 1
-  const int per = S / kVTile;
-  const int cl = (nvt + per - 1) / per;
-  if (cl > kMaxCl || (long long)rows * cl > 0x7fffffffLL) return cudaErrorNotSupported;
-  const size_t smem = smem_bytes(S) + (size_t)cl * kG * kD * sizeof(float);
+template <typename T, int S>
+cudaError_t run_slice(const DecodeArgs& a, int rows, int cl, cudaStream_t stream) {
   static bool attr_set = false;  // benign race: every caller sets the same value
   if (!attr_set) {
-    const size_t max_smem = smem_bytes(4096) + (size_t)kMaxCl * kG * kD * sizeof(float);
     const cudaError_t e =
-        cudaFuncSetAttribute(k_decode_mma<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_smem);
+        cudaFuncSetAttribute(k_decode_mma<T, S>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes(S));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(rows * cl), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = smem_bytes(S);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -462,7 +475,18 @@ cudaError_t run(const DecodeArgs& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_decode_mma<T>, a, cl, S);
+  return cudaLaunchKernelEx(&cfg, k_decode_mma<T, S>, a, cl);
+}
+
+template <typename T>
+cudaError_t run(const DecodeArgs& a, cudaStream_t stream) {
+  const int rows = a.B * a.Hkv;
+  const int nvt = (a.n + kVTile - 1) / kVTile;
+  const bool small = nvt <= kMaxCl * (2048 / kVTile);  // n <= 16384: 3 CTAs per SM
+  const int per = (small ? 2048 : 4096) / kVTile;
+  const int cl = (nvt + per - 1) / per;
+  if (cl > kMaxCl || (long long)rows * cl > 0x7fffffffLL) return cudaErrorNotSupported;
+  return small ? run_slice<T, 2048>(a, rows, cl, stream) : run_slice<T, 4096>(a, rows, cl, stream);
 }
 
 }  // namespace
