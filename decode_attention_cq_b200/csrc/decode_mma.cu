@@ -50,6 +50,8 @@ constexpr int kPartStride = kD + 8;  // floats per (warp pair, head) row of the 
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Fixed {
+  // raw rows (dtype T) staged first: q of the 4 heads, alpha_K, s_K, alpha_V, s_V
+  alignas(16) uint8_t stage[8 * kD * 4];
   uint8_t limb[kG * 3][kLimbRow];  // K-side weight limbs: row 3 h + l, byte = channel
   float red[kWarps][kG][2];        // per-warp reduction scratch
   float mM[kMaxCl][kG][2];         // every peer's logit range per head (pushed to all)
@@ -151,8 +153,21 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1) k_decode_mma(Deco
   const int nunits = (t1 - t0 + kUnit - 1) / kUnit;  // K units of this CTA
   const uint32_t sK_u = tc::smem_u32(sK), sV_u = tc::smem_u32(sV);
 
-  // ---- 1. stream this slice's codes into shared memory (K first, then V)
+  // ---- 1. stream the query and statistics rows, then this slice's codes into
+  // shared memory (three cp.async groups: rows, K codes, V codes)
   {
+    constexpr int kRowChunks = kD * (int)sizeof(T) / 16;  // 16-byte chunks per row
+    const uint8_t* qrow = static_cast<const uint8_t*>(a.q) + ((size_t)b * a.Hq + (size_t)kG * hkv) * kD * sizeof(T);
+    const size_t stat = (size_t)row * kD * sizeof(T);
+    const uint8_t* srcs[4] = {static_cast<const uint8_t*>(a.k_alpha) + stat, static_cast<const uint8_t*>(a.k_scale) + stat,
+                              static_cast<const uint8_t*>(a.v_alpha) + stat, static_cast<const uint8_t*>(a.v_scale) + stat};
+    const uint32_t st_u = tc::smem_u32(F.stage);
+    for (int e = t; e < 8 * kRowChunks; e += kThreads) {
+      const int r = e / kRowChunks, c = e % kRowChunks;
+      const uint8_t* src = r < kG ? qrow + (size_t)e * 16 : srcs[r - kG] + (size_t)c * 16;
+      cp_async16(st_u + e * 16, src, true);
+    }
+    cp_async_commit();
     const uint8_t* kc = a.k_codes + (size_t)row * octets * kD;
     const int oct0 = t0 / 8;
     for (int e = t; e < nunits * 16 * 8; e += kThreads) {  // 16-byte chunks of K
@@ -172,14 +187,16 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1) k_decode_mma(Deco
   tc::cluster_arrive_relaxed();  // matched by the wait before the first peer store
 
   // ---- 2. post-scaled K weights w_h = sigma q_h (.) s_K in 22-bit fixed point
+  const T* sRows = reinterpret_cast<const T*>(F.stage);  // q[4][kD], alpha_K, s_K, alpha_V, s_V
+  cp_async_wait<2>();
+  __syncthreads();
   float w[kG];
   if (t < kD) {
-    const T* qp = static_cast<const T*>(a.q) + ((size_t)b * a.Hq + (size_t)kG * hkv) * kD;
-    const float sk = DT<T>::f(static_cast<const T*>(a.k_scale)[(size_t)row * kD + t]);
-    const float ak = DT<T>::f(static_cast<const T*>(a.k_alpha)[(size_t)row * kD + t]);
+    const float ak = DT<T>::f(sRows[4 * kD + t]);
+    const float sk = DT<T>::f(sRows[5 * kD + t]);
 #pragma unroll
     for (int h = 0; h < kG; ++h) {
-      const float qv = DT<T>::f(qp[h * kD + t]);
+      const float qv = DT<T>::f(sRows[h * kD + t]);
       w[h] = a.sigma * qv * sk;
       const float amax = warp_max(fabsf(w[h]));
       const float qa = warp_sum(qv * ak);
@@ -255,8 +272,8 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1) k_decode_mma(Deco
         const float sc = kscale * __int_as_float((127 - k - kk) << 23);  // step * 2^-k
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          const float v = fmaf(16384.f, (float)d[kk][1][2 * r],
-                               fmaf(128.f, (float)d[kk][0][2 * r + 1], (float)d[kk][0][2 * r]));
+          const int d01 = d[kk][0][2 * r] + (d[kk][0][2 * r + 1] << 7);  // |d01| < 2^29
+          const float v = fmaf(16384.f, (float)d[kk][1][2 * r], (float)d01);
           const float x = fmaf(v, sc, c0);
           if (tok + 64 * r + k + kk < t1) {
             mn = fminf(mn, x);
@@ -445,9 +462,8 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1) k_decode_mma(Deco
         s += F.recv[(r * kG + h) * wrecv + ch - first];
         l += F.part_l[r][h];
       }
-      const size_t kv = (size_t)row * kD + ch;
-      const float alpha = DT<T>::f(static_cast<const T*>(a.v_alpha)[kv]);
-      const float step = DT<T>::f(static_cast<const T*>(a.v_scale)[kv]);
+      const float alpha = DT<T>::f(sRows[6 * kD + ch]);
+      const float step = DT<T>::f(sRows[7 * kD + ch]);
       T* out = static_cast<T*>(a.out) + ((size_t)b * a.Hq + (size_t)kG * hkv + h) * kD;
       out[ch] = DT<T>::from_float(fmaf(step, s / l, alpha));
     }
