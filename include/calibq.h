@@ -189,7 +189,10 @@ cq_status cq_decode_attn_workspace_size(cq_layout k_layout, cq_layout v_layout, 
  *
  * Supported layout pairs: (CANONICAL, CANONICAL) for any bits and any Hq/Hkv;
  * (OCTET_K, OCTET_V) for bits = 1, d = 128, Hq = 4*Hkv and n <= 65536 -- the
- * tensor-core path.
+ * tensor-core path (register-fed MMAs up to n = 32768, tcgen05 beyond; setting
+ * the environment variable CALIBQ_DECODE_KERNEL=tcgen05 before the first call
+ * selects tcgen05 for every n). Results of the two kernels agree within the
+ * output tolerance, not bit for bit.
  */
 cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, const void* k_alpha,
                          const void* k_scale, cq_layout k_layout, const uint8_t* v_codes,

@@ -1,0 +1,38 @@
+"""Both octet-layout decode kernels against the fp64 oracle: the mma.sync
+kernel (default up to n = 32768) and the tcgen05 kernel (rows longer than
+that, or every row when CALIBQ_DECODE_KERNEL=tcgen05), each in a child process
+so that the selection, read once per process, applies."""
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+from _util import OUT_RTOL
+
+pytestmark = pytest.mark.gpu
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+CASES = [[1, 1, [True, 0.8, 0.9]], [300, 2, [False, 1.0, 1.0]], [1025, 2, [True, 0.8, 0.9]],
+         [2049, 1, [True, 1.0, 0.5]], [8192, 1, [True, 0.8, 0.9]], [10000, 1, [True, 0.5, 1.0]],
+         [12000, 1, [True, 0.8, 0.9]], [14000, 1, [True, 0.8, 0.9]], [20000, 1, [True, 0.8, 0.9]]]
+
+
+def _run(kernel):
+    env = dict(os.environ)
+    env.pop("CALIBQ_DECODE_KERNEL", None)
+    if kernel:
+        env["CALIBQ_DECODE_KERNEL"] = kernel
+    res = subprocess.run([sys.executable, os.path.join(HERE, "_kernel_select_worker.py"), json.dumps(CASES)],
+                         env=env, capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
+    return json.loads(res.stdout.strip().splitlines()[-1])["errs"]
+
+
+@pytest.mark.parametrize("kernel", [None, "tcgen05"])
+def test_octet_kernels_match_oracle(cuda_device, kernel):
+    errs = _run(kernel)
+    for (n, batch, calib), e in zip(CASES, errs):
+        assert e <= OUT_RTOL, (kernel, n, calib, e)
