@@ -27,6 +27,7 @@
 //  6. sums the warps, scatters the (head, channel) partial sums over the
 //     cluster so that every CTA owns a range of channels, and writes o.
 // Everything stays on chip; one launch per decode step, no workspace.
+#include <cuda.h>  // CUtensorMap (encoded through the runtime's driver entry point; no libcuda link)
 #include <float.h>
 
 #include "common.cuh"
@@ -48,10 +49,15 @@ constexpr int kLimbRow = 132;  // bytes per limb row (padding spreads the B-frag
 constexpr int kRecv = kG * 136;  // >= kG * cl * ceil(kD / cl) for every cl <= 8
 constexpr int kPartStride = kD + 8;  // floats per (warp pair, head) row of the partial sums
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kKBoxRows = 128;      // octet rows per K tensor-copy box (8 units, 16 KB)
+constexpr int kMaxKBoxes = 4;       // 4096-token slices
+constexpr uint32_t kSpin = 1u << 24;  // bound on every mbarrier wait (about a second)
 
 struct Fixed {
   // raw rows (dtype T) staged first: q of the 4 heads, alpha_K, s_K, alpha_V, s_V
   alignas(16) uint8_t stage[8 * kD * 4];
+  uint64_t bar_rows, bar_v, bar_k[kMaxKBoxes];  // copy completion, one phase per launch
+  int err;                                      // a bounded wait ran out
   uint8_t limb[kG * 3][kLimbRow];  // K-side weight limbs: row 3 h + l, byte = channel
   float red[kWarps][kG][2];        // per-warp reduction scratch
   float mM[kMaxCl][kG][2];         // every peer's logit range per head (pushed to all)
@@ -65,16 +71,6 @@ struct Fixed {
 // (S/8 x 128 B) | V codes / partial sums (S/256 x 4 KB) | fixed part.
 __host__ __device__ constexpr size_t smem_bytes(int slice) {
   return (size_t)slice / 8 * 128 + (size_t)slice / kVTile * 4096 + sizeof(Fixed);
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
@@ -130,10 +126,23 @@ __device__ __forceinline__ int logit_pos(int unit, int k, int h, int o) {
   return (((k * kG + h) ^ (unit & 1)) << 4) + (o ^ ((h >> 1) << 3));
 }
 
+// Every thread waits for the copy phase; a wait that runs out flags the CTA
+// (its outputs become NaN) instead of hanging.
+__device__ __forceinline__ void wait_copies(uint64_t* bar, volatile int* err) {
+  if (!tc::mbar_wait(bar, 0, kSpin)) *err = 1;
+}
+
+// kmap: K codes as [rows][octets][128 B], 128-byte swizzle (16-byte chunk c of
+// octet row r lands at chunk c ^ (r & 7)); vmap: V codes as [rows * tiles][128
+// channels][32 B], 32-byte swizzle (half h of channel row ch lands at half
+// h ^ ((ch >> 2) & 1)). Both swizzles make the ldmatrix reads conflict-free.
 template <typename T, int S>
-__global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1) k_decode_mma(DecodeArgs a, int cl) {
+__global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
+    k_decode_mma(const __grid_constant__ DecodeArgs a, int cl, const __grid_constant__ CUtensorMap kmap,
+                 const __grid_constant__ CUtensorMap vmap) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* sK = smem_raw;                      // [S/8][128] codes, 16-byte chunks swizzled by octet
+  // the 128-byte swizzle of the K copies repeats every 1024 bytes: align to it
+  uint8_t* sK = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);                      // [S/8][128] codes, 16-byte chunks swizzled by octet
   uint8_t* sV = sK + (size_t)S / 8 * 128;      // [S/256][128][32] codes, halves swizzled by channel
   Fixed& F = *reinterpret_cast<Fixed*>(sV + (size_t)S / kVTile * 4096);
   float* sL = reinterpret_cast<float*>(sK);    // logits, unit u at floats [512 u, 512 u + 512)
@@ -145,7 +154,6 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1) k_decode_mma(Deco
   const int row = blockIdx.x / cl;
   const int b = row / a.Hkv, hkv = row % a.Hkv;
   const int n = a.n;
-  const int octets = (n + 7) >> 3;
   const int nvt = (n + kVTile - 1) / kVTile;
   const int vt0 = (int)((rank * nvt) / cl), vt1 = (int)(((rank + 1) * nvt) / cl);
   const int t0 = vt0 * kVTile, t1 = min(n, vt1 * kVTile);
@@ -153,43 +161,39 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1) k_decode_mma(Deco
   const int nunits = (t1 - t0 + kUnit - 1) / kUnit;  // K units of this CTA
   const uint32_t sK_u = tc::smem_u32(sK), sV_u = tc::smem_u32(sV);
 
-  // ---- 1. stream the query and statistics rows, then this slice's codes into
-  // shared memory (three cp.async groups: rows, K codes, V codes)
-  {
-    constexpr int kRowChunks = kD * (int)sizeof(T) / 16;  // 16-byte chunks per row
-    const uint8_t* qrow = static_cast<const uint8_t*>(a.q) + ((size_t)b * a.Hq + (size_t)kG * hkv) * kD * sizeof(T);
-    const size_t stat = (size_t)row * kD * sizeof(T);
-    const uint8_t* srcs[4] = {static_cast<const uint8_t*>(a.k_alpha) + stat, static_cast<const uint8_t*>(a.k_scale) + stat,
-                              static_cast<const uint8_t*>(a.v_alpha) + stat, static_cast<const uint8_t*>(a.v_scale) + stat};
-    const uint32_t st_u = tc::smem_u32(F.stage);
-    for (int e = t; e < 8 * kRowChunks; e += kThreads) {
-      const int r = e / kRowChunks, c = e % kRowChunks;
-      const uint8_t* src = r < kG ? qrow + (size_t)e * 16 : srcs[r - kG] + (size_t)c * 16;
-      cp_async16(st_u + e * 16, src, true);
+  // ---- 1. one thread streams the query and statistics rows, then this slice's
+  // codes into shared memory with bulk / tensor copies (no per-thread copy
+  // instructions stand in the way of the other warps' shared-memory traffic)
+  const int nkbox = (nunits * 16 + kKBoxRows - 1) / kKBoxRows;  // K boxes of 8 units
+  volatile int* err = &F.err;
+  if (t == 0) {
+    F.err = 0;
+    tc::mbar_init(&F.bar_rows, 1);
+    tc::mbar_init(&F.bar_v, 1);
+    for (int i = 0; i < kMaxKBoxes; ++i) tc::mbar_init(&F.bar_k[i], 1);
+    tc::fence_mbar_init();
+    constexpr uint32_t kRow = kD * sizeof(T);
+    const uint8_t* qrow = static_cast<const uint8_t*>(a.q) + ((size_t)b * a.Hq + (size_t)kG * hkv) * kRow;
+    const size_t stat = (size_t)row * kRow;
+    tc::mbar_arrive_expect_tx(&F.bar_rows, 8 * kRow);
+    tc::bulk_load(F.stage, qrow, kG * kRow, &F.bar_rows);
+    tc::bulk_load(F.stage + 4 * kRow, static_cast<const uint8_t*>(a.k_alpha) + stat, kRow, &F.bar_rows);
+    tc::bulk_load(F.stage + 5 * kRow, static_cast<const uint8_t*>(a.k_scale) + stat, kRow, &F.bar_rows);
+    tc::bulk_load(F.stage + 6 * kRow, static_cast<const uint8_t*>(a.v_alpha) + stat, kRow, &F.bar_rows);
+    tc::bulk_load(F.stage + 7 * kRow, static_cast<const uint8_t*>(a.v_scale) + stat, kRow, &F.bar_rows);
+    for (int i = 0; i < nkbox; ++i) {  // octet rows past the row's end arrive as zeros
+      tc::mbar_arrive_expect_tx(&F.bar_k[i], kKBoxRows * 128);
+      tc::tma_load_3d(sK + (size_t)i * kKBoxRows * 128, &kmap, 0, t0 / 8 + i * kKBoxRows, row, &F.bar_k[i]);
     }
-    cp_async_commit();
-    const uint8_t* kc = a.k_codes + (size_t)row * octets * kD;
-    const int oct0 = t0 / 8;
-    for (int e = t; e < nunits * 16 * 8; e += kThreads) {  // 16-byte chunks of K
-      const int lo = e >> 3, c16 = e & 7, oct = oct0 + lo;
-      const bool ok = oct < octets;
-      cp_async16(sK_u + lo * 128 + ((c16 ^ (lo & 7)) << 4), kc + (size_t)(ok ? oct : 0) * kD + c16 * 16, ok);
-    }
-    cp_async_commit();
-    const uint8_t* vc = a.v_codes + (size_t)row * nvt * 4096 + (size_t)vt0 * 4096;
-    for (int e = t; e < nvtl * 256; e += kThreads) {  // 16-byte chunks of V
-      const int tile = e >> 8, ch = (e >> 1) & 127, half = e & 1;
-      cp_async16(sV_u + tile * 4096 + ch * 32 + ((half ^ ((ch >> 2) & 1)) << 4),
-                 vc + (size_t)tile * 4096 + ch * 32 + half * 16, true);
-    }
-    cp_async_commit();
+    tc::mbar_arrive_expect_tx(&F.bar_v, (uint32_t)nvtl * 4096);
+    for (int i = 0; i < nvtl; ++i) tc::tma_load_3d(sV + (size_t)i * 4096, &vmap, 0, 0, row * nvt + vt0 + i, &F.bar_v);
   }
   tc::cluster_arrive_relaxed();  // matched by the wait before the first peer store
+  __syncthreads();               // barrier initialisation is visible
 
   // ---- 2. post-scaled K weights w_h = sigma q_h (.) s_K in 22-bit fixed point
   const T* sRows = reinterpret_cast<const T*>(F.stage);  // q[4][kD], alpha_K, s_K, alpha_V, s_V
-  cp_async_wait<2>();
-  __syncthreads();
+  wait_copies(&F.bar_rows, err);
   float w[kG];
   if (t < kD) {
     const float ak = DT<T>::f(sRows[4 * kD + t]);
@@ -237,11 +241,11 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1) k_decode_mma(Deco
     }
   const float c0 = F.c0[tq], kscale = F.kscale[tq];
 
-  // ---- 3. K side: warp w takes units w, w + 8, ...; per unit 16 octets x 128 channels
-  cp_async_wait<1>();  // this thread's K chunks have landed
-  __syncthreads();     // ... and everybody else's
+  // ---- 3. K side: warp w takes units w, w + 8, ... (unit w + 8 i is in copy box i);
+  // per unit 16 octets x 128 channels
   float mn = FLT_MAX, mx = -FLT_MAX;  // logit range of head tq over this lane's tokens
   for (int u = warp; u < nunits; u += kWarps) {
+    wait_copies(&F.bar_k[u / kWarps], err);
     uint32_t af[4][4];  // A fragments of chunks c = 0..3 (rows = octets 16u + {g, g+8})
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
@@ -376,8 +380,8 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1) k_decode_mma(Deco
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
     if (grp == 0) F.lsum[warp][h] = lsum;
   }
-  cp_async_wait<0>();  // V codes
-  __syncthreads();
+  wait_copies(&F.bar_v, err);
+  __syncthreads();  // the weight fragments are complete
 
   // ---- 6. V side: warp pair p = warp / 2 takes tiles p, p + 4, ...; warp parity
   // picks channels 64 hc .. 64 hc + 63. D rows (limb, head), columns channels.
@@ -463,26 +467,67 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1) k_decode_mma(Deco
         l += F.part_l[r][h];
       }
       const float alpha = DT<T>::f(sRows[6 * kD + ch]);
-      const float step = DT<T>::f(sRows[7 * kD + ch]);
+      const float step = *err ? __int_as_float(0x7fc00000) : DT<T>::f(sRows[7 * kD + ch]);
       T* out = static_cast<T*>(a.out) + ((size_t)b * a.Hq + (size_t)kG * hkv + h) * kD;
       out[ch] = DT<T>::from_float(fmaf(step, s / l, alpha));
     }
   }
+  if (*err && t == 0) {  // let copies still in flight land before the CTA's memory is reused
+    tc::mbar_wait(&F.bar_rows, 0, kSpin);
+    tc::mbar_wait(&F.bar_v, 0, kSpin);
+    for (int i = 0; i < nkbox; ++i) tc::mbar_wait(&F.bar_k[i], 0, kSpin);
+  }
+}
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<EncodeTiled>(p);
+  }();
+  return fn;
+}
+
+// 3-D uint8 map {inner bytes, mid, outer} with box {inner, box_mid, 1}.
+bool encode_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer, uint32_t box_mid,
+               CUtensorMapSwizzle swz) {
+  const EncodeTiled fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {inner, mid, outer};
+  const cuuint64_t strides[2] = {inner, inner * mid};
+  const cuuint32_t box[3] = {(cuuint32_t)inner, box_mid, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <typename T, int S>
 cudaError_t run_slice(const DecodeArgs& a, int rows, int cl, cudaStream_t stream) {
+  const size_t smem = smem_bytes(S) + 1024;  // slack to align the codes to the 1024-byte swizzle atom
   static bool attr_set = false;  // benign race: every caller sets the same value
   if (!attr_set) {
     const cudaError_t e =
-        cudaFuncSetAttribute(k_decode_mma<T, S>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes(S));
+        cudaFuncSetAttribute(k_decode_mma<T, S>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
+  const int octets = (a.n + 7) / 8, nvt = (a.n + kVTile - 1) / kVTile;
+  CUtensorMap kmap, vmap;
+  if (!encode_3d(&kmap, a.k_codes, kD, (uint64_t)octets, (uint64_t)rows, kKBoxRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_3d(&vmap, a.v_codes, 32, kD, (uint64_t)rows * nvt, kD, CU_TENSOR_MAP_SWIZZLE_32B))
+    return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(rows * cl), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem_bytes(S);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -491,7 +536,7 @@ cudaError_t run_slice(const DecodeArgs& a, int rows, int cl, cudaStream_t stream
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_decode_mma<T, S>, a, cl);
+  return cudaLaunchKernelEx(&cfg, k_decode_mma<T, S>, a, cl, kmap, vmap);
 }
 
 template <typename T>
