@@ -358,12 +358,21 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
         const float xs[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
         const int i0 = t0 + lt * kVTile + 32 * grp + k;  // token of j = 0
         uint32_t P[4];
+        if (t0 + (lt + 1) * kVTile <= t1) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const bool ok = i0 + 8 * j < t1;
-          const float p = ex2_approx(fmaf(xs[j], alog2, bias));
-          P[j] = ok ? __float2uint_rn(p) : 0u;
-          lsum += ok ? p * unscale : 0.f;
+          for (int j = 0; j < 4; ++j) {
+            const float p = ex2_approx(fmaf(xs[j], alog2, bias));
+            P[j] = __float2uint_rn(p);
+            lsum += p;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const bool ok = i0 + 8 * j < t1;
+            const float p = ex2_approx(fmaf(xs[j], alog2, bias));
+            P[j] = ok ? __float2uint_rn(p) : 0u;
+            lsum += ok ? p : 0.f;
+          }
         }
         // word l = byte l of P[0..3]
         const uint32_t lo01 = __byte_perm(P[0], P[1], 0x5140), hi01 = __byte_perm(P[0], P[1], 0x7362);
@@ -374,6 +383,7 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
         *reinterpret_cast<uint2*>(dst + (size_t)lt * 4096 + 256) = make_uint2(w1, w3);
       }
     }
+    lsum *= unscale;
     // lanes with equal h: xor over grp
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
