@@ -9,8 +9,9 @@
 //
 // One thread-block cluster per (batch, kv-head) row, one CTA per slice of at
 // most S tokens (S = 2048, or 4096 for n > 16384). Each CTA
-//  1. streams its slice of K and V codes into shared memory with cp.async
-//     (16-byte chunks, XOR-swizzled so that ldmatrix reads are conflict-free);
+//  1. streams its slice of K and V codes into shared memory with a few tensor
+//     copies issued by one thread (128-byte swizzle, so that ldmatrix reads are
+//     conflict-free), completing on mbarriers;
 //  2. K side: per unit of 16 token octets (128 tokens) a warp loads the A
 //     fragments of all 128 channels with ldmatrix; masking bit k of every byte
 //     gives "code of token 8 r + k times 2^k" for octet row r. B holds the
@@ -51,6 +52,7 @@ constexpr int kPartStride = kD + 8;  // floats per (warp pair, head) row of the 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kKBoxRows = 128;      // octet rows per K tensor-copy box (8 units, 16 KB)
 constexpr int kMaxKBoxes = 4;       // 4096-token slices
+constexpr int kVBoxLines = 256;     // 128-byte V lines per tensor-copy box (8 tiles, 32 KB)
 constexpr uint32_t kSpin = 1u << 24;  // bound on every mbarrier wait (about a second)
 
 struct Fixed {
@@ -132,10 +134,10 @@ __device__ __forceinline__ void wait_copies(uint64_t* bar, volatile int* err) {
   if (!tc::mbar_wait(bar, 0, kSpin)) *err = 1;
 }
 
-// kmap: K codes as [rows][octets][128 B], 128-byte swizzle (16-byte chunk c of
-// octet row r lands at chunk c ^ (r & 7)); vmap: V codes as [rows * tiles][128
-// channels][32 B], 32-byte swizzle (half h of channel row ch lands at half
-// h ^ ((ch >> 2) & 1)). Both swizzles make the ldmatrix reads conflict-free.
+// kmap: K codes as [rows][octets][128 B]; vmap: V codes as [rows][tiles * 32][128 B]
+// (a 128-byte line holds 4 channels' 32 bytes of a tile). Both use the 128-byte
+// swizzle: 16-byte chunk c of line l lands at chunk c ^ (l & 7), which keeps
+// every ldmatrix phase on 32 distinct banks.
 template <typename T, int S>
 __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
     k_decode_mma(const __grid_constant__ DecodeArgs a, int cl, const __grid_constant__ CUtensorMap kmap,
@@ -143,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the 128-byte swizzle of the K copies repeats every 1024 bytes: align to it
   uint8_t* sK = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);                      // [S/8][128] codes, 16-byte chunks swizzled by octet
-  uint8_t* sV = sK + (size_t)S / 8 * 128;      // [S/256][128][32] codes, halves swizzled by channel
+  uint8_t* sV = sK + (size_t)S / 8 * 128;      // [S/256 tiles][32 lines][128 B] codes, swizzled
   Fixed& F = *reinterpret_cast<Fixed*>(sV + (size_t)S / kVTile * 4096);
   float* sL = reinterpret_cast<float*>(sK);    // logits, unit u at floats [512 u, 512 u + 512)
   uint8_t* sFrag = sK;                         // weight-limb A fragments, tile lt at bytes [4096 lt, ...)
@@ -185,8 +187,10 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
       tc::mbar_arrive_expect_tx(&F.bar_k[i], kKBoxRows * 128);
       tc::tma_load_3d(sK + (size_t)i * kKBoxRows * 128, &kmap, 0, t0 / 8 + i * kKBoxRows, row, &F.bar_k[i]);
     }
-    tc::mbar_arrive_expect_tx(&F.bar_v, (uint32_t)nvtl * 4096);
-    for (int i = 0; i < nvtl; ++i) tc::tma_load_3d(sV + (size_t)i * 4096, &vmap, 0, 0, row * nvt + vt0 + i, &F.bar_v);
+    const int nvbox = (nvtl * 32 + kVBoxLines - 1) / kVBoxLines;  // lines past the row's end arrive as zeros
+    tc::mbar_arrive_expect_tx(&F.bar_v, (uint32_t)nvbox * kVBoxLines * 128);
+    for (int i = 0; i < nvbox; ++i)
+      tc::tma_load_3d(sV + (size_t)i * kVBoxLines * 128, &vmap, 0, vt0 * 32 + i * kVBoxLines, row, &F.bar_v);
   }
   tc::cluster_arrive_relaxed();  // matched by the wait before the first peer store
   __syncthreads();               // barrier initialisation is visible
@@ -407,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
       const int mat = lane >> 3, half = mat & 1;
       const int ch = 64 * hc + 16 * p + 8 * (mat >> 1) + (lane & 7);
       uint32_t r[4];
-      ldsm_x4(tile_u + ch * 32 + ((half ^ ((ch >> 2) & 1)) << 4), r);
+      ldsm_x4(tile_u + (ch >> 2) * 128 + (((((ch & 3) << 1) | half) ^ ((ch >> 2) & 7)) << 4), r);
       bv[2 * p][0] = r[0];
       bv[2 * p][1] = r[1];
       bv[2 * p + 1][0] = r[2];
@@ -532,7 +536,7 @@ cudaError_t run_slice(const DecodeArgs& a, int rows, int cl, cudaStream_t stream
   const int octets = (a.n + 7) / 8, nvt = (a.n + kVTile - 1) / kVTile;
   CUtensorMap kmap, vmap;
   if (!encode_3d(&kmap, a.k_codes, kD, (uint64_t)octets, (uint64_t)rows, kKBoxRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_3d(&vmap, a.v_codes, 32, kD, (uint64_t)rows * nvt, kD, CU_TENSOR_MAP_SWIZZLE_32B))
+      !encode_3d(&vmap, a.v_codes, 128, (uint64_t)nvt * 32, (uint64_t)rows, kVBoxLines, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(rows * cl), 1, 1);
