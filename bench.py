@@ -67,15 +67,15 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def traffic_record(path: str):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel
-    source has not changed since it was captured."""
+def traffic_record(path: str, workload: str, bits: int):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    this workload and the kernel source has not changed since."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         rec = json.load(f).get(path)
-    if not rec:
+    if not rec or rec.get("workload") != workload or rec.get("bits", 1) != bits:
         return None
     src = os.path.join(ROOT, DECODE_KERNEL_SOURCES[path])
     digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
@@ -279,7 +279,7 @@ def run_ours(args, world, rank, local):
     alg = algorithmic_bytes(B, w.hq, w.hkv, n, w.d, bits)
     kernel_ms = sum(step_ms) / len(step_ms)  # one launch per step on the octet path
     achieved = alg / (kernel_ms * 1e-3) / 1e9
-    trec = traffic_record(args.path)
+    trec = traffic_record(args.path, args.workload, bits)
     fill_mean = sum(fill_ms) / len(fill_ms)
     fill_alg = cache_fill_bytes(B, w.hkv, n, w.d, bits)
     line = {
