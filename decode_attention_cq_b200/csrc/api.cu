@@ -67,16 +67,14 @@ cq_status check_shape(int B, int H, int n, int d, int bits) {
 }
 
 cq_status row_bytes(cq_layout layout, int n, int bits, size_t* out) {
-  if (!valid_layout(layout)) return CQ_ERR_INVALID_ARG;
+  if (!valid_layout(layout) || !valid_bits(bits)) return CQ_ERR_INVALID_ARG;
   switch (layout) {
     case CQ_LAYOUT_CANONICAL: *out = (size_t)n * kD * bits / 8; return CQ_OK;
-    case CQ_LAYOUT_OCTET_K:
-      if (bits != 1) return CQ_ERR_UNSUPPORTED;
-      *out = (size_t)((n + 7) / 8) * kD;
+    case CQ_LAYOUT_OCTET_K:  // 8 / bits tokens per byte
+      *out = (size_t)((n + 8 / bits - 1) / (8 / bits)) * kD;
       return CQ_OK;
-    default:
-      if (bits != 1) return CQ_ERR_UNSUPPORTED;
-      *out = (size_t)((n + 255) / 256) * 4096;
+    default:  // tiles of 256 / bits tokens
+      *out = (size_t)((n + 256 / bits - 1) / (256 / bits)) * 4096;
       return CQ_OK;
   }
 }

@@ -15,12 +15,13 @@ __device__ __forceinline__ int read_code(const uint8_t* row, cq_layout layout, i
   if (layout == CQ_LAYOUT_CANONICAL) {
     byte = (size_t)i * (kD * BITS / 8) + (j * BITS) / 8;
     bit = (j * BITS) % 8;
-  } else if (layout == CQ_LAYOUT_OCTET_K) {
-    byte = (size_t)(i >> 3) * kD + j;
-    bit = i & 7;
-  } else {
-    byte = (size_t)(i >> 8) * 4096 + j * 32 + ((i & 255) >> 3);
-    bit = i & 7;
+  } else if (layout == CQ_LAYOUT_OCTET_K) {  // P = 8 / BITS tokens per byte
+    byte = (size_t)(i / (8 / BITS)) * kD + j;
+    bit = (i % (8 / BITS)) * BITS;
+  } else {  // tiles of 32 P tokens
+    constexpr int kTile = 32 * (8 / BITS);
+    byte = (size_t)(i / kTile) * 4096 + j * 32 + (i % kTile) / (8 / BITS);
+    bit = (i % (8 / BITS)) * BITS;
   }
   return (row[byte] >> bit) & ((1 << BITS) - 1);
 }
@@ -45,8 +46,8 @@ cudaError_t run(const uint8_t* codes, const T* alpha, const T* scale, cq_layout 
                 int n, int bits, T* out, cudaStream_t stream) {
   size_t row_bytes;
   if (layout == CQ_LAYOUT_CANONICAL) row_bytes = (size_t)n * kD * bits / 8;
-  else if (layout == CQ_LAYOUT_OCTET_K) row_bytes = (size_t)((n + 7) / 8) * kD;
-  else row_bytes = (size_t)((n + 255) / 256) * 4096;
+  else if (layout == CQ_LAYOUT_OCTET_K) row_bytes = (size_t)((n + 8 / bits - 1) / (8 / bits)) * kD;
+  else row_bytes = (size_t)((n + 256 / bits - 1) / (256 / bits)) * 4096;
   const dim3 grid((unsigned)(((size_t)n * kD + 255) / 256), rows);
   switch (bits) {
     case 1: k_dequant<T, 1><<<grid, 256, 0, stream>>>(codes, alpha, scale, layout, n, row_bytes, out); break;

@@ -205,6 +205,87 @@ __global__ void __launch_bounds__(kThreads) k_pack_octet_v(
   }
 }
 
+// OCTET_K layout with BITS in {2, 4, 8}: P = 8 / BITS tokens share a byte; a
+// thread owns one byte group (P tokens) x 8 channels, i.e. 8 consecutive bytes.
+template <typename T, int BITS>
+__global__ void __launch_bounds__(kThreads) k_pack_octet_k_b(
+    const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
+    uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
+  constexpr int L = (1 << BITS) - 1, P = 8 / BITS;
+  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
+  const int row = blockIdx.x;
+  fold_stats<T>(part, row, S, L, s_alpha, s_beta, s_inv, alpha_out, scale_out);
+  const int cb = threadIdx.x % kTpr, r = threadIdx.x / kTpr;
+  float af[8], inv[8];
+  double ad[8], bd[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    af[e] = s_alpha[cb * 8 + e];
+    inv[e] = s_inv[cb * 8 + e];
+    ad[e] = (double)af[e];
+    bd[e] = (double)s_beta[cb * 8 + e];
+  }
+  const int groups = (n + P - 1) / P;
+  const int m0 = blockIdx.y * (tile_tokens / P), m1 = min(groups, m0 + tile_tokens / P);
+  const T* xr = x + (size_t)row * n * kD + cb * 8;
+  uint8_t* cr = codes + (size_t)row * groups * kD + cb * 8;
+  for (int m = m0 + r; m < m1; m += kRpi) {
+    uint64_t bytes = 0;
+#pragma unroll
+    for (int k = 0; k < P; ++k) {
+      const int i = P * m + k;
+      if (i < n) {
+        float v[8];
+        load8(xr + (size_t)i * kD, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          bytes |= (uint64_t)quant_code(v[e], af[e], inv[e], ad[e], bd[e], L) << (8 * e + BITS * k);
+      }
+    }
+    *reinterpret_cast<uint64_t*>(cr + (size_t)m * kD) = bytes;
+  }
+}
+
+// OCTET_V layout with BITS in {2, 4, 8}: tiles of 32 P tokens; byte column q of
+// a tile holds tokens P q .. P q + P - 1. A warp owns one tile: lane q builds
+// byte column q of every channel (consecutive lanes write consecutive bytes).
+template <typename T, int BITS>
+__global__ void __launch_bounds__(kThreads) k_pack_octet_v_b(
+    const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
+    uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
+  constexpr int L = (1 << BITS) - 1, P = 8 / BITS, kTile = 32 * P;
+  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
+  const int row = blockIdx.x;
+  fold_stats<T>(part, row, S, L, s_alpha, s_beta, s_inv, alpha_out, scale_out);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tiles = (n + kTile - 1) / kTile;
+  const int v0 = blockIdx.y * (tile_tokens / kTile), v1 = min(tiles, v0 + tile_tokens / kTile);
+  const T* xr = x + (size_t)row * n * kD;
+  uint8_t* cr = codes + (size_t)row * tiles * 4096;
+  for (int vt = v0 + warp; vt < v1; vt += kThreads / 32) {
+#pragma unroll 1
+    for (int cg = 0; cg < kD / 8; ++cg) {
+      uint32_t bytes[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+      for (int k = 0; k < P; ++k) {
+        const int i = vt * kTile + P * lane + k;
+        if (i < n) {
+          float v[8];
+          load8(xr + (size_t)i * kD + cg * 8, v);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int j = cg * 8 + e;
+            bytes[e] |= (uint32_t)quant_code(v[e], s_alpha[j], s_inv[j], (double)s_alpha[j], (double)s_beta[j], L)
+                        << (BITS * k);
+          }
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cr[(size_t)vt * 4096 + (cg * 8 + e) * 32 + lane] = (uint8_t)bytes[e];
+    }
+  }
+}
+
 }  // namespace
 
 int quantize_splits(int rows, int n) {
@@ -232,13 +313,23 @@ static cudaError_t launch_quantize_t(const T* x, int rows, int n, int bits, cq_l
       default: k_pack_canonical<T, 8><<<grid, kThreads, 0, stream>>>(x, n, S, tile, part, codes, alpha, scale); break;
     }
   } else if (layout == CQ_LAYOUT_OCTET_K) {
-    const int n_pad = (n + 7) / 8 * 8;
-    k_pack_octet_k<T><<<dim3(rows, (n_pad + tile - 1) / tile), kThreads, 0, stream>>>(
-        x, n, S, tile, part, codes, alpha, scale);
+    const int P = 8 / bits, n_pad = (n + P - 1) / P * P;
+    const dim3 grid(rows, (n_pad + tile - 1) / tile);
+    switch (bits) {
+      case 1: k_pack_octet_k<T><<<grid, kThreads, 0, stream>>>(x, n, S, tile, part, codes, alpha, scale); break;
+      case 2: k_pack_octet_k_b<T, 2><<<grid, kThreads, 0, stream>>>(x, n, S, tile, part, codes, alpha, scale); break;
+      case 4: k_pack_octet_k_b<T, 4><<<grid, kThreads, 0, stream>>>(x, n, S, tile, part, codes, alpha, scale); break;
+      default: k_pack_octet_k_b<T, 8><<<grid, kThreads, 0, stream>>>(x, n, S, tile, part, codes, alpha, scale); break;
+    }
   } else {
-    const int n_pad = (n + 255) / 256 * 256;
-    k_pack_octet_v<T><<<dim3(rows, (n_pad + tile - 1) / tile), kThreads, 0, stream>>>(
-        x, n, S, tile, part, codes, alpha, scale);
+    const int vtile = 32 * (8 / bits), n_pad = (n + vtile - 1) / vtile * vtile;
+    const dim3 grid(rows, (n_pad + tile - 1) / tile);
+    switch (bits) {
+      case 1: k_pack_octet_v<T><<<grid, kThreads, 0, stream>>>(x, n, S, tile, part, codes, alpha, scale); break;
+      case 2: k_pack_octet_v_b<T, 2><<<grid, kThreads, 0, stream>>>(x, n, S, tile, part, codes, alpha, scale); break;
+      case 4: k_pack_octet_v_b<T, 4><<<grid, kThreads, 0, stream>>>(x, n, S, tile, part, codes, alpha, scale); break;
+      default: k_pack_octet_v_b<T, 8><<<grid, kThreads, 0, stream>>>(x, n, S, tile, part, codes, alpha, scale); break;
+    }
   }
   return cudaGetLastError();
 }

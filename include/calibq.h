@@ -56,17 +56,22 @@ typedef enum cq_dtype { CQ_F16 = 0, CQ_F32 = 1 } cq_dtype;
  *   little-endian bit string, i.e. at bit (j*bits) % 32 of little-endian
  *   uint32 word (j*bits)/32 of the token.
  *
- * CQ_LAYOUT_OCTET_K (bits = 1, d = 128; row_bytes = ceil(n/8) * 128):
- *   one byte per (8 consecutive tokens, channel). Token i, channel j:
- *       byte = (i >> 3) * 128 + j,        bit = i & 7.
- *   (Row m of the [n/8][128] byte matrix is one tensor-memory lane of the
- *   K-side tensor-core operand; masking bit k of every byte selects token
- *   8m + k.)
+ * CQ_LAYOUT_OCTET_K (bits in {1, 2, 4, 8}, d = 128; P = 8 / bits tokens share
+ *   a byte; row_bytes = ceil(n/P) * 128): one byte per (P consecutive tokens,
+ *   channel). Token i, channel j:
+ *       byte = (i / P) * 128 + j,         code at bits [(i % P) * bits, +bits).
+ *   For bits = 1: byte = (i >> 3) * 128 + j, bit = i & 7. (Row m of the
+ *   [n/P][128] byte matrix is one row of the K-side tensor-core operand;
+ *   masking sub-position k of every byte gives "code of token P m + k times
+ *   2^(k bits)" as an 8-bit operand.)
  *
- * CQ_LAYOUT_OCTET_V (bits = 1, d = 128; row_bytes = ceil(n/256) * 4096):
- *   the same bytes, transposed per tile of 256 tokens. Token i, channel j:
- *       byte = (i >> 8) * 4096 + j * 32 + ((i & 255) >> 3),   bit = i & 7.
- *   (Channel j's 32 bytes of a tile are one tensor-memory lane of the V-side
+ * CQ_LAYOUT_OCTET_V (bits in {1, 2, 4, 8}, d = 128; row_bytes =
+ *   ceil(n / (32 P)) * 4096): the same bytes, transposed per tile of 32 P
+ *   tokens (256 for bits = 1). Token i, channel j:
+ *       byte = (i / (32 P)) * 4096 + j * 32 + (i % (32 P)) / P,
+ *       code at bits [(i % P) * bits, +bits).
+ *   For bits = 1: byte = (i >> 8) * 4096 + j * 32 + ((i & 255) >> 3), bit =
+ *   i & 7. (Channel j's 32 bytes of a tile are one column of the V-side
  *   operand.)
  *
  * Padding tokens (n..padded-1) of the octet layouts hold code 0 and are

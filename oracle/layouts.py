@@ -10,15 +10,17 @@ position and packs / unpacks with that map, one bit at a time.
   d*b/8 consecutive bytes; channel j's code sits at bits [j*b, j*b + b) of the
   token's little-endian bit string, i.e. byte (j*b) // 8, bits (j*b) % 8 ...
 
-* octet-K (b = 1, d = 128): byte-per-(8 tokens, channel). Token i,
-  channel j:   byte = (i >> 3) * 128 + j,   bit = i & 7.
-  Row bytes = ceil(n / 8) * 128.
+* octet-K (b in {1, 2, 4, 8}, d = 128): one byte per (P = 8/b consecutive
+  tokens, channel). Token i, channel j:
+      byte = (i // P) * 128 + j,   bit = (i % P) * b.
+  Row bytes = ceil(n / P) * 128. (b = 1: byte (i >> 3) * 128 + j, bit i & 7.)
 
-* octet-V (b = 1, d = 128): the same bytes transposed per 256-token tile.
-  Token i, channel j:   byte = (i >> 8) * 4096 + j * 32 + ((i & 255) >> 3),
-  bit = i & 7.   Row bytes = ceil(n / 256) * 4096.
+* octet-V (b in {1, 2, 4, 8}, d = 128): the same bytes transposed per tile of
+  32 P tokens. Token i, channel j:
+      byte = (i // (32 P)) * 4096 + j * 32 + (i % (32 P)) // P,   bit = (i % P) * b.
+  Row bytes = ceil(n / (32 P)) * 4096. (b = 1: 256-token tiles.)
 
-Tokens past n in the last octet / tile are padding and hold code 0.
+Tokens past n in the last byte group / tile are padding and hold code 0.
 """
 
 from __future__ import annotations
@@ -29,32 +31,39 @@ LAYOUT_CANONICAL = 0
 LAYOUT_OCTET_K = 1
 LAYOUT_OCTET_V = 2
 
-_TILE = {LAYOUT_OCTET_K: 8, LAYOUT_OCTET_V: 256}
+def _per_byte(bits: int) -> int:
+    """Tokens sharing one byte of an octet layout."""
+    return 8 // bits
+
+
+def _tile(layout: int, bits: int) -> int:
+    """Tokens of one padding unit: a byte group (octet-K) or a tile (octet-V)."""
+    return _per_byte(bits) * (32 if layout == LAYOUT_OCTET_V else 1)
 
 
 def _check(layout: int, d: int, bits: int):
     if layout == LAYOUT_CANONICAL:
         if (d * bits) % 32:
             raise ValueError("canonical layout needs d*bits to be a multiple of 32")
-    elif layout in _TILE:
-        if bits != 1 or d != 128:
-            raise ValueError("octet layouts are defined for bits=1, d=128")
+    elif layout in (LAYOUT_OCTET_K, LAYOUT_OCTET_V):
+        if bits not in (1, 2, 4, 8) or d != 128:
+            raise ValueError("octet layouts are defined for bits in {1, 2, 4, 8}, d=128")
     else:
         raise ValueError(f"unknown layout {layout}")
 
 
-def padded_tokens(layout: int, n: int) -> int:
-    """Tokens stored per row: n, or n rounded up to the layout's tile."""
+def padded_tokens(layout: int, n: int, bits: int = 1) -> int:
+    """Tokens stored per row: n, or n rounded up to the layout's padding unit."""
     if layout == LAYOUT_CANONICAL:
         return n
-    t = _TILE[layout]
+    t = _tile(layout, bits)
     return -(-n // t) * t
 
 
 def codes_nbytes(layout: int, n: int, d: int, bits: int) -> int:
     """Bytes of one (batch, head) row of packed codes."""
     _check(layout, d, bits)
-    return padded_tokens(layout, n) * d * bits // 8
+    return padded_tokens(layout, n, bits) * d * bits // 8
 
 
 def bit_position(layout: int, i, j, n: int, d: int, bits: int):
@@ -69,10 +78,12 @@ def bit_position(layout: int, i, j, n: int, d: int, bits: int):
         row = d * bits // 8
         pos = j * bits
         return i * row + pos // 8, pos % 8
+    p = _per_byte(bits)
     if layout == LAYOUT_OCTET_K:
-        return (i >> 3) * 128 + j, i & 7
+        return (i // p) * 128 + j, (i % p) * bits
     # LAYOUT_OCTET_V
-    return (i >> 8) * 4096 + j * 32 + ((i & 255) >> 3), i & 7
+    tile = 32 * p
+    return (i // tile) * 4096 + j * 32 + (i % tile) // p, (i % p) * bits
 
 
 def pack_codes(codes, layout: int, bits: int) -> np.ndarray:

@@ -48,7 +48,9 @@ def test_version_and_status_strings(lib):
 
 
 @pytest.mark.parametrize("layout,bits,n", [(0, 1, 3328), (0, 2, 5), (0, 8, 8192), (1, 1, 3328),
-                                           (1, 1, 9), (2, 1, 3328), (2, 1, 8192), (2, 1, 1)])
+                                           (1, 1, 9), (2, 1, 3328), (2, 1, 8192), (2, 1, 1),
+                                           (1, 2, 3329), (2, 2, 3329), (1, 4, 7), (2, 4, 65),
+                                           (1, 8, 1), (2, 8, 33)])
 def test_codes_bytes_match_the_documented_layouts(lib, layout, bits, n):
     B, H = 3, 2
     assert cq.cq_codes_bytes(layout, B, H, n, 128, bits) == B * H * oracle.codes_nbytes(layout, n, 128, bits)
@@ -56,7 +58,7 @@ def test_codes_bytes_match_the_documented_layouts(lib, layout, bits, n):
 
 def test_size_queries_validate(lib):
     with pytest.raises(cq.CalibqError) as e:
-        cq.cq_codes_bytes(1, 1, 1, 16, 128, 2)  # octet layouts are 1-bit only
+        cq.cq_codes_bytes(1, 1, 1, 16, 64, 2)  # octet layouts need d = 128
     assert e.value.status == cq.CQ_ERR_UNSUPPORTED
     with pytest.raises(cq.CalibqError) as e:
         cq.cq_codes_bytes(0, 1, 1, 16, 64, 1)

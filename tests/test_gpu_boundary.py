@@ -35,7 +35,8 @@ def test_quantize_rejections(cuda_device):
     assert call(args(x=x.data_ptr() + 2)) == cq.CQ_ERR_INVALID_ARG          # misaligned
     assert call(args(nws=ws.numel() - 1)) == cq.CQ_ERR_WORKSPACE            # small workspace
     assert call(args(ws=None)) == cq.CQ_ERR_WORKSPACE
-    assert call(args(), layout=1, bits=2) == cq.CQ_ERR_UNSUPPORTED          # octet needs 1 bit
+    assert call(args(), layout=1, bits=3) == cq.CQ_ERR_INVALID_ARG          # bits not in {1, 2, 4, 8}
+    assert call(args(), layout=7, bits=1) == cq.CQ_ERR_INVALID_ARG          # unknown layout
     torch.cuda.synchronize()
     assert torch.equal(qc.codes, sentinel)
 

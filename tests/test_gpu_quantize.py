@@ -66,6 +66,19 @@ def test_octet_codes_bit_exact(cuda_device, dtype, layout, n):
     _check_quantized(x, qc, 1, LAYOUTS[layout])
 
 
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+@pytest.mark.parametrize("layout", ["octet_k", "octet_v"])
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("n", [1, 3, 31, 33, 64, 65, 129, 1000, 2049])
+def test_octet_multibit_codes_bit_exact(cuda_device, dtype, layout, bits, n):
+    """b-bit octet layouts (8/b tokens per byte): ragged tails inside a byte
+    group and inside a V tile of 256/b tokens."""
+    x = _cache(2, 2, n, dtype, seed=1000 * bits + n)
+    qc = cq.cq_quantize_kv(x.to(cuda_device), bits, LAYOUTS[layout])
+    torch.cuda.synchronize()
+    _check_quantized(x, qc, bits, LAYOUTS[layout])
+
+
 def test_exact_ties_and_constant_channels(cuda_device):
     """Inputs that sit exactly on rounding ties and channels with beta == alpha."""
     n = 64
@@ -75,7 +88,7 @@ def test_exact_ties_and_constant_channels(cuda_device):
         x[0, 0, :, c] = torch.arange(n, dtype=torch.float32) * (0.25 + (c % 5)) - (c % 7)
     x[0, 1] = 3.5  # every channel constant
     for bits in (1, 2, 4, 8):
-        for layout in (cq.LAYOUT_CANONICAL,) + ((cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V) if bits == 1 else ()):
+        for layout in (cq.LAYOUT_CANONICAL, cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V):
             qc = cq.cq_quantize_kv(x.to(cuda_device), bits, layout)
             torch.cuda.synchronize()
             ref = _check_quantized(x, qc, bits, layout)
@@ -84,7 +97,7 @@ def test_exact_ties_and_constant_channels(cuda_device):
 
 @pytest.mark.parametrize("layout", ["canonical", "octet_k", "octet_v"])
 def test_dequant_matches_oracle(cuda_device, layout):
-    bits_list = [1, 2, 4, 8] if layout == "canonical" else [1]
+    bits_list = [1, 2, 4, 8]
     for dtype in ("f16", "f32"):
         for bits in bits_list:
             x = _cache(1, 2, 333, dtype, seed=bits + 3)

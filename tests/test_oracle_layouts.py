@@ -27,7 +27,7 @@ def _rows():
 
 def test_hand_worked_positions():
     rows = _rows()
-    assert len(rows) >= 18
+    assert len(rows) >= 32
     for layout, bits, d, i, j, byte, bit in rows:
         n = i + 1
         got = oracle.bit_position(layout, i, j, n, d, bits)
@@ -42,7 +42,10 @@ def test_hand_worked_positions():
 
 @pytest.mark.parametrize("layout,bits,n", [(LAYOUT_CANONICAL, 1, 37), (LAYOUT_CANONICAL, 2, 5),
                                            (LAYOUT_CANONICAL, 4, 9), (LAYOUT_CANONICAL, 8, 3),
-                                           (LAYOUT_OCTET_K, 1, 300), (LAYOUT_OCTET_V, 1, 300)])
+                                           (LAYOUT_OCTET_K, 1, 300), (LAYOUT_OCTET_V, 1, 300),
+                                           (LAYOUT_OCTET_K, 2, 301), (LAYOUT_OCTET_V, 2, 301),
+                                           (LAYOUT_OCTET_K, 4, 99), (LAYOUT_OCTET_V, 4, 99),
+                                           (LAYOUT_OCTET_K, 8, 45), (LAYOUT_OCTET_V, 8, 45)])
 def test_positions_are_a_bijection_onto_the_row(layout, bits, n):
     d = 128
     ii, jj = np.meshgrid(np.arange(n), np.arange(d), indexing="ij")
@@ -52,12 +55,14 @@ def test_positions_are_a_bijection_onto_the_row(layout, bits, n):
     nbytes = oracle.codes_nbytes(layout, n, d, bits)
     assert flat.min() >= 0 and flat.max() < nbytes * 8
     # padding bits of the octet layouts are exactly the unused tail
-    assert nbytes * 8 == oracle.padded_tokens(layout, n) * d * bits
+    assert nbytes * 8 == oracle.padded_tokens(layout, n, bits) * d * bits
 
 
 @pytest.mark.parametrize("layout,bits,n", [(LAYOUT_CANONICAL, 1, 77), (LAYOUT_CANONICAL, 2, 33),
                                            (LAYOUT_CANONICAL, 8, 11), (LAYOUT_OCTET_K, 1, 257),
-                                           (LAYOUT_OCTET_V, 1, 513)])
+                                           (LAYOUT_OCTET_V, 1, 513), (LAYOUT_OCTET_K, 2, 130),
+                                           (LAYOUT_OCTET_V, 4, 200), (LAYOUT_OCTET_K, 8, 33),
+                                           (LAYOUT_OCTET_V, 8, 70)])
 def test_pack_unpack_round_trip(layout, bits, n):
     rng = np.random.default_rng(n)
     codes = rng.integers(0, 1 << bits, size=(2, 3, n, 128))
@@ -110,9 +115,26 @@ def test_octet_v_rows_are_tensor_memory_a_rows():
                     assert (int(got[0]), int(got[1])) == want
 
 
+def test_octet_sub_positions_are_tensor_operand_values():
+    """b bits: masking sub-position k of every byte ((2^b - 1) << k b) gives the
+    8-bit operand "code of token P m + k times 2^(k b)" for byte group m, and
+    (2^b - 1) << k b never exceeds 255."""
+    for bits in (2, 4, 8):
+        p = 8 // bits
+        rng = np.random.default_rng(bits)
+        n = 4 * p
+        codes = rng.integers(0, 1 << bits, size=(1, 1, n, 128))
+        packed = oracle.pack_codes(codes, LAYOUT_OCTET_K, bits)[0, 0].reshape(-1, 128)
+        for m in range(n // p):
+            for k in range(p):
+                mask = ((1 << bits) - 1) << (k * bits)
+                assert mask <= 255
+                assert np.array_equal(packed[m] & mask, codes[0, 0, p * m + k] << (k * bits))
+
+
 def test_layout_arguments_are_checked():
     with pytest.raises(ValueError):
-        oracle.codes_nbytes(LAYOUT_OCTET_K, 10, 128, 2)
+        oracle.codes_nbytes(LAYOUT_OCTET_K, 10, 128, 3)
     with pytest.raises(ValueError):
         oracle.codes_nbytes(LAYOUT_OCTET_V, 10, 64, 1)
     with pytest.raises(ValueError):
