@@ -188,7 +188,8 @@ cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, con
   if (!generic && !octet) return CQ_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;
   if (generic && G > 32) return CQ_ERR_UNSUPPORTED;
-  if (octet && (G != 4 || bits != 1 || n > 65536)) return CQ_ERR_UNSUPPORTED;
+  if (octet && (G != 4 || (bits == 1 ? n > 65536 : !cq::decode_ring_supports(n, bits))))
+    return CQ_ERR_UNSUPPORTED;
   const void* ptrs[] = {q, k_codes, k_alpha, k_scale, v_codes, v_alpha, v_scale, out};
   for (const void* p : ptrs) CQ_TRY(check_ptr(p));
   cq::DecodeArgs a;
@@ -216,9 +217,9 @@ cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, con
     CQ_TRY(check_ptr(workspace));
     return cuda_status(cq::launch_decode_generic(a, dt, workspace, s));
   }
-  const cudaError_t e = (cq::decode_mma_supports(n) && !force_tcgen05())
-                            ? cq::launch_decode_mma(a, dt, s)
-                            : cq::launch_decode_octet(a, dt, s);
+  const cudaError_t e = bits != 1 ? cq::launch_decode_ring(a, dt, s)
+                        : (cq::decode_mma_supports(n) && !force_tcgen05()) ? cq::launch_decode_mma(a, dt, s)
+                                                                            : cq::launch_decode_octet(a, dt, s);
   if (e == cudaErrorNotSupported) return CQ_ERR_UNSUPPORTED;
   return cuda_status(e);
 }

@@ -28,20 +28,21 @@
 //  6. sums the warps, scatters the (head, channel) partial sums over the
 //     cluster so that every CTA owns a range of channels, and writes o.
 // Everything stays on chip; one launch per decode step, no workspace.
-#include <cuda.h>  // CUtensorMap (encoded through the runtime's driver entry point; no libcuda link)
 #include <float.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "mma_util.cuh"
 #include "tc.cuh"
 
 namespace cq {
 
 namespace {
 
+using namespace mu;
+
 constexpr int kThreads = 256;  // 8 warps
 constexpr int kWarps = kThreads / 32;
-constexpr int kG = 4;          // query heads per kv-head
 constexpr int kUnit = 128;     // tokens per K-side unit (16 octets, 2 KB of codes)
 constexpr int kVTile = 256;    // tokens per V-side tile (32 octets, 4 KB of codes)
 constexpr int kMaxCl = 8;
@@ -53,7 +54,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kKBoxRows = 128;      // octet rows per K tensor-copy box (8 units, 16 KB)
 constexpr int kMaxKBoxes = 4;       // 4096-token slices
 constexpr int kVBoxLines = 256;     // 128-byte V lines per tensor-copy box (8 tiles, 32 KB)
-constexpr uint32_t kSpin = 1u << 24;  // bound on every mbarrier wait (about a second)
 
 struct Fixed {
   // raw rows (dtype T) staged first: q of the 4 heads, alpha_K, s_K, alpha_V, s_V
@@ -73,65 +73,6 @@ struct Fixed {
 // (S/8 x 128 B) | V codes / partial sums (S/256 x 4 KB) | fixed part.
 __host__ __device__ constexpr size_t smem_bytes(int slice) {
   return (size_t)slice / 8 * 128 + (size_t)slice / kVTile * 4096 + sizeof(Fixed);
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr)
-               : "memory");
-}
-__device__ __forceinline__ void lds128(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr)
-               : "memory");
-}
-
-// D += A (16x32 u8, row) x B (32x8 s8, col). Register-only: the compiler may
-// interleave independent MMAs.
-__device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-// D += A (16x32 u8, row) x B (32x8 u8, col)
-__device__ __forceinline__ void mma_u8u8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-// Position (in floats, within its unit's 2 KB) of the logit of octet o (0..15)
-// of a unit, bit position k, head h. Rows of 16 floats; odd units swap row
-// pairs and heads 2, 3 swap octet halves, so that both the K-side stores and
-// the softmax-side float4 loads are free of bank conflicts.
-__device__ __forceinline__ int logit_pos(int unit, int k, int h, int o) {
-  return (((k * kG + h) ^ (unit & 1)) << 4) + (o ^ ((h >> 1) << 3));
-}
-
-// Every thread waits for the copy phase; a wait that runs out flags the CTA
-// (its outputs become NaN) instead of hanging.
-__device__ __forceinline__ void wait_copies(uint64_t* bar, volatile int* err) {
-  if (!tc::mbar_wait(bar, 0, kSpin)) *err = 1;
 }
 
 // kmap: K codes as [rows][octets][128 B]; vmap: V codes as [rows][tiles * 32][128 B]
@@ -197,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
 
   // ---- 2. post-scaled K weights w_h = sigma q_h (.) s_K in 22-bit fixed point
   const T* sRows = reinterpret_cast<const T*>(F.stage);  // q[4][kD], alpha_K, s_K, alpha_V, s_V
-  wait_copies(&F.bar_rows, err);
+  wait_copies(&F.bar_rows, 0, err);
   float w[kG];
   if (t < kD) {
     const float ak = DT<T>::f(sRows[4 * kD + t]);
@@ -249,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
   // per unit 16 octets x 128 channels
   float mn = FLT_MAX, mx = -FLT_MAX;  // logit range of head tq over this lane's tokens
   for (int u = warp; u < nunits; u += kWarps) {
-    wait_copies(&F.bar_k[u / kWarps], err);
+    wait_copies(&F.bar_k[u / kWarps], 0, err);
     uint32_t af[4][4];  // A fragments of chunks c = 0..3 (rows = octets 16u + {g, g+8})
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
@@ -394,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
     if (grp == 0) F.lsum[warp][h] = lsum;
   }
-  wait_copies(&F.bar_v, err);
+  wait_copies(&F.bar_v, 0, err);
   __syncthreads();  // the weight fragments are complete
 
   // ---- 6. V side: warp pair p = warp / 2 takes tiles p, p + 4, ...; warp parity
@@ -491,36 +432,6 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
     tc::mbar_wait(&F.bar_v, 0, kSpin);
     for (int i = 0; i < nkbox; ++i) tc::mbar_wait(&F.bar_k[i], 0, kSpin);
   }
-}
-
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encode_fn() {
-  static EncodeTiled fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      p = nullptr;
-    return reinterpret_cast<EncodeTiled>(p);
-  }();
-  return fn;
-}
-
-// 3-D uint8 map {inner bytes, mid, outer} with box {inner, box_mid, 1}.
-bool encode_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer, uint32_t box_mid,
-               CUtensorMapSwizzle swz) {
-  const EncodeTiled fn = encode_fn();
-  if (fn == nullptr) return false;
-  const cuuint64_t dims[3] = {inner, mid, outer};
-  const cuuint64_t strides[2] = {inner, inner * mid};
-  const cuuint32_t box[3] = {(cuuint32_t)inner, box_mid, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <typename T, int S>

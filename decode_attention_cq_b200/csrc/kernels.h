@@ -48,6 +48,10 @@ cudaError_t launch_decode_generic(const DecodeArgs& a, cq_dtype dt, void* worksp
 // ---- decode_octet.cu (octet layouts, bits = 1, Hq = 4 Hkv, tensor cores)
 cudaError_t launch_decode_octet(const DecodeArgs& a, cq_dtype dt, cudaStream_t stream);
 
+// ---- decode_ring.cu (octet layouts, bits in {2, 4, 8}, Hq = 4 Hkv, n <= 32768, mma.sync)
+bool decode_ring_supports(int n, int bits);
+cudaError_t launch_decode_ring(const DecodeArgs& a, cq_dtype dt, cudaStream_t stream);
+
 // ---- decode_mma.cu (octet layouts, bits = 1, Hq = 4 Hkv, n <= 32768, mma.sync)
 bool decode_mma_supports(int n);
 cudaError_t launch_decode_mma(const DecodeArgs& a, cq_dtype dt, cudaStream_t stream);
