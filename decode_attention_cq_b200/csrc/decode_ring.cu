@@ -17,7 +17,8 @@
 // One thread-block cluster per (batch, kv-head) row, one CTA per 2048-token
 // slice, whatever b is. Only the slice's logits (later its weight fragments,
 // 16 bytes per token) stay resident; the codes (32 b KB per slice for K and
-// again for V) stream through a two-slot ring of 16 KB tensor copies: K
+// again for V) stream through a ring of 16 KB tensor copies (2 slots, 4 for
+// 4- and 8-bit codes): K
 // chunks first, then V chunks, so the first V chunks load while the cluster
 // exchanges the logit range. A slot is refilled once all eight warps have
 // released it (full / empty mbarriers, every wait bounded).
@@ -50,7 +51,7 @@ template <typename T>
 struct RingFixed {
   // raw rows (dtype T): q of the 4 heads, alpha_K, s_K, alpha_V, s_V
   alignas(16) uint8_t stage[8 * kD * sizeof(T)];
-  uint64_t bar_rows, full[2], empty[2];
+  uint64_t bar_rows, full[4], empty[4];
   int err;                          // a bounded wait ran out
   uint8_t limb[kG * 3][kLimbRow];   // K-side weight limbs: row 3 h + l, byte = channel
   float red[kWarps][kG][2];         // per-warp reduction scratch
@@ -61,17 +62,23 @@ struct RingFixed {
   float recv[kRecv];                // [src][h][channel - first owned channel]
 };
 
-// logits / weight fragments (16 B per token) | ring (2 x 16 KB) | fixed part
-template <typename T>
+// Ring slots: 2 (3 CTAs per SM) while the K / V loops have work to hide the
+// copies behind; 4 (2 CTAs per SM, more bytes in flight per SM) for 4- and
+// 8-bit codes, where the kernel mostly waits on its copies.
+template <int BITS>
+constexpr int ring_slots() { return BITS >= 4 ? 4 : 2; }
+
+// logits / weight fragments (16 B per token) | ring (slots x 16 KB) | fixed part
+template <typename T, int BITS>
 constexpr size_t ring_smem_bytes() {
-  return (size_t)kSlice * 16 + 2 * kChunkBytes + sizeof(RingFixed<T>);
+  return (size_t)kSlice * 16 + (size_t)ring_slots<BITS>() * kChunkBytes + sizeof(RingFixed<T>);
 }
 
 // kmap: K codes as [rows][byte rows][128 B]; vmap: V codes as [rows][tiles *
 // 32][128 B] (a 128-byte line holds 4 channels' 32 bytes of a tile). Both use
 // the 128-byte swizzle (chunk c of line l lands at chunk c ^ (l & 7)).
 template <typename T, int BITS>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, ring_slots<BITS>() == 2 ? 3 : 2)
     k_decode_ring(const __grid_constant__ DecodeArgs a, int cl, const __grid_constant__ CUtensorMap kmap,
                   const __grid_constant__ CUtensorMap vmap) {
   constexpr int P = 8 / BITS;         // tokens per code byte
@@ -79,12 +86,13 @@ __global__ void __launch_bounds__(kThreads, 3)
   constexpr int kTileTok = 32 * P;    // tokens per V tile (32 byte columns, 4 KB)
   constexpr int kUnitWords = 64 * P;  // logit words per unit (16 byte rows x P x 4 heads)
   constexpr uint32_t kSubMask = 0x01010101u * ((1u << BITS) - 1u);  // sub-position 0 of every byte
+  constexpr int kSlots = ring_slots<BITS>();
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the 128-byte swizzle of the copies repeats every 1024 bytes: align to it
   uint8_t* sL = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* ring = sL + (size_t)kSlice * 16;
-  RingFixed<T>& F = *reinterpret_cast<RingFixed<T>*>(ring + 2 * kChunkBytes);
+  RingFixed<T>& F = *reinterpret_cast<RingFixed<T>*>(ring + kSlots * kChunkBytes);
   float* sLf = reinterpret_cast<float*>(sL);   // logits, unit u at words [kUnitWords u, ...)
   float* sPart = reinterpret_cast<float*>(ring);  // per warp-pair partial sums (after the V side)
   const uint32_t sL_u = tc::smem_u32(sL), ring_u = tc::smem_u32(ring);
@@ -104,22 +112,22 @@ __global__ void __launch_bounds__(kThreads, 3)
   const int nchunks = nk + nv;
   volatile int* err = &F.err;
 
-  // chunk gi of the ring sequence (K chunks, then V chunks) into slot gi % 2;
+  // chunk gi of the ring sequence (K chunks, then V chunks) into slot gi % kSlots;
   // rows past the row's end arrive as zeros
   auto issue = [&](int gi) {
-    const int slot = gi & 1;
+    const int slot = gi % kSlots;
     tc::mbar_arrive_expect_tx(&F.full[slot], kChunkBytes);
     if (gi < nk)
       tc::tma_load_3d(ring + slot * kChunkBytes, &kmap, 0, t0 / P + gi * kChunkRows, row, &F.full[slot]);
     else
       tc::tma_load_3d(ring + slot * kChunkBytes, &vmap, 0, vt0 * 32 + (gi - nk) * kChunkRows, row, &F.full[slot]);
   };
-  // after every warp released slot gi % 2 (chunk gi): refill it with chunk gi + 2
+  // after every warp released the slot of chunk gi: refill it with chunk gi + kSlots
   auto refill = [&](int gi) {
-    if (t == 0 && gi + 2 < nchunks) {
-      if (tc::mbar_wait(&F.empty[gi & 1], ((uint32_t)gi >> 1) & 1u, kSpin)) {
+    if (t == 0 && gi + kSlots < nchunks) {
+      if (tc::mbar_wait(&F.empty[gi % kSlots], (uint32_t)(gi / kSlots) & 1u, kSpin)) {
         tc::fence_proxy_async();
-        issue(gi + 2);
+        issue(gi + kSlots);
       } else {
         *err = 1;
       }
@@ -130,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, 3)
   if (t == 0) {
     F.err = 0;
     tc::mbar_init(&F.bar_rows, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kSlots; ++i) {
       tc::mbar_init(&F.full[i], 1);
       tc::mbar_init(&F.empty[i], kWarps);
     }
@@ -144,8 +152,7 @@ __global__ void __launch_bounds__(kThreads, 3)
     tc::bulk_load(F.stage + 5 * kRow, static_cast<const uint8_t*>(a.k_scale) + stat, kRow, &F.bar_rows);
     tc::bulk_load(F.stage + 6 * kRow, static_cast<const uint8_t*>(a.v_alpha) + stat, kRow, &F.bar_rows);
     tc::bulk_load(F.stage + 7 * kRow, static_cast<const uint8_t*>(a.v_scale) + stat, kRow, &F.bar_rows);
-    issue(0);
-    if (nchunks > 1) issue(1);
+    for (int gi = 0; gi < kSlots && gi < nchunks; ++gi) issue(gi);
   }
   tc::cluster_arrive_relaxed();  // matched by the wait before the first peer store
   __syncthreads();               // barrier initialisation is visible
@@ -205,8 +212,8 @@ __global__ void __launch_bounds__(kThreads, 3)
   constexpr int KK = P >= 2 ? 2 : 1;  // sub-positions per pass (independent accumulators)
   float mn = FLT_MAX, mx = -FLT_MAX;  // logit range of head tq over this lane's tokens
   for (int gk = 0; gk < nk; ++gk) {
-    const int slot = gk & 1;
-    wait_copies(&F.full[slot], ((uint32_t)gk >> 1) & 1u, err);
+    const int slot = gk % kSlots;
+    wait_copies(&F.full[slot], (uint32_t)(gk / kSlots) & 1u, err);
     const int u = kWarps * gk + warp;
     if (u < nunits) {
       uint32_t af[4][4];  // A fragments of chunks c = 0..3 (rows = byte rows {g, g+8} of the unit)
@@ -367,8 +374,8 @@ __global__ void __launch_bounds__(kThreads, 3)
 #pragma unroll
   for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0;
   for (int gv = 0; gv < nv; ++gv) {
-    const int gi = nk + gv, slot = gi & 1;
-    wait_copies(&F.full[slot], ((uint32_t)gi >> 1) & 1u, err);
+    const int gi = nk + gv, slot = gi % kSlots;
+    wait_copies(&F.full[slot], (uint32_t)(gi / kSlots) & 1u, err);
     const int lt = 4 * gv + pair;
     if (lt < nvtl) {
       const uint32_t tile_u = ring_u + slot * kChunkBytes + pair * 4096;
@@ -460,8 +467,8 @@ __global__ void __launch_bounds__(kThreads, 3)
   }
   if (*err && t == 0) {  // let copies still in flight land before the CTA's memory is reused
     tc::mbar_wait(&F.bar_rows, 0, kSpin);
-    for (int gi = nchunks - 2; gi < nchunks; ++gi)
-      if (gi >= 0) tc::mbar_wait(&F.full[gi & 1], ((uint32_t)gi >> 1) & 1u, kSpin);
+    for (int gi = nchunks - kSlots; gi < nchunks; ++gi)
+      if (gi >= 0) tc::mbar_wait(&F.full[gi % kSlots], (uint32_t)(gi / kSlots) & 1u, kSpin);
   }
 }
 
@@ -473,7 +480,7 @@ cudaError_t run_bits(const DecodeArgs& a, cudaStream_t stream) {
   const int per = kSlice / kTileTok;  // V tiles per CTA
   const int cl = (nvt + per - 1) / per;
   if (cl > kMaxCl || (long long)rows * cl > 0x7fffffffLL) return cudaErrorNotSupported;
-  const size_t smem = ring_smem_bytes<T>() + 1024;  // slack to align to the 1024-byte swizzle atom
+  const size_t smem = ring_smem_bytes<T, BITS>() + 1024;  // slack to align to the 1024-byte swizzle atom
   static bool attr_set = false;  // benign race: every caller sets the same values
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(k_decode_ring<T, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
