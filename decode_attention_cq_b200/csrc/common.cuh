@@ -71,4 +71,20 @@ __device__ __forceinline__ int quant_code(float xf, float af, float inv, double 
   return inv > 0.f ? c : 0;
 }
 
+// 1-bit codes: with L = 1 the rounding rule above reduces to code = [x - alpha >
+// (beta - alpha) / 2] = [2x > alpha + beta] (a tie gives 0, as round-half-to-
+// even of 1/2 does; a constant channel gives 0). With alpha + beta held as the
+// exact pair s_hi + s_lo (two_sum), the float test fl(2x - s_hi) > s_lo is exact:
+// when 2x and s_hi are within a factor of two the subtraction is exact
+// (Sterbenz); otherwise |2x - s_hi| >= |s_hi| / 2 > |s_lo| and rounding cannot
+// move it across s_lo.
+__device__ __forceinline__ void two_sum(float a, float b, float& hi, float& lo) {
+  hi = __fadd_rn(a, b);
+  const float t = __fsub_rn(hi, a);
+  lo = __fadd_rn(__fsub_rn(a, __fsub_rn(hi, t)), __fsub_rn(b, t));
+}
+__device__ __forceinline__ uint32_t code1(float x, float s_hi, float s_lo) {
+  return __fmaf_rn(2.f, x, -s_hi) > s_lo ? 1u : 0u;
+}
+
 }  // namespace cq

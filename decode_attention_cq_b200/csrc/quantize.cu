@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(kThreads) k_pack_canonical(
   const int row = blockIdx.x;
   fold_stats<T>(part, row, S, L, s_alpha, s_beta, s_inv, alpha_out, scale_out);
   const int cg = threadIdx.x % kTpr, r = threadIdx.x / kTpr;
-  float af[8], inv[8];
+  float af[8], inv[8], hi[8], lo[8];
   double ad[8], bd[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(kThreads) k_pack_canonical(
     inv[e] = s_inv[cg * 8 + e];
     ad[e] = (double)af[e];
     bd[e] = (double)s_beta[cg * 8 + e];
+    two_sum(af[e], s_beta[cg * 8 + e], hi[e], lo[e]);  // used for 1-bit codes
   }
   const int i0 = blockIdx.y * tile_tokens, i1 = min(n, i0 + tile_tokens);
   const T* xr = x + (size_t)row * n * kD + cg * 8;
@@ -114,8 +115,12 @@ __global__ void __launch_bounds__(kThreads) k_pack_canonical(
     load8(xr + (size_t)i * kD, v);
     uint64_t packed = 0;
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      packed |= (uint64_t)quant_code(v[e], af[e], inv[e], ad[e], bd[e], L) << (e * BITS);
+    for (int e = 0; e < 8; ++e) {
+      if constexpr (BITS == 1)
+        packed |= (uint64_t)code1(v[e], hi[e], lo[e]) << e;
+      else
+        packed |= (uint64_t)quant_code(v[e], af[e], inv[e], ad[e], bd[e], L) << (e * BITS);
+    }
     uint8_t* dst = cr + (size_t)i * (kD * BITS / 8);
     if (BITS == 1) *dst = (uint8_t)packed;
     if (BITS == 2) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
@@ -134,15 +139,9 @@ __global__ void __launch_bounds__(kThreads) k_pack_octet_k(
   const int row = blockIdx.x;
   fold_stats<T>(part, row, S, 1, s_alpha, s_beta, s_inv, alpha_out, scale_out);
   const int cb = threadIdx.x % kTpr, r = threadIdx.x / kTpr;
-  float af[8], inv[8];
-  double ad[8], bd[8];
+  float hi[8], lo[8];  // alpha + beta of the thread's channels as an exact pair
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    af[e] = s_alpha[cb * 8 + e];
-    inv[e] = s_inv[cb * 8 + e];
-    ad[e] = (double)af[e];
-    bd[e] = (double)s_beta[cb * 8 + e];
-  }
+  for (int e = 0; e < 8; ++e) two_sum(s_alpha[cb * 8 + e], s_beta[cb * 8 + e], hi[e], lo[e]);
   const int octets = (n + 7) / 8;
   const int m0 = blockIdx.y * (tile_tokens / 8), m1 = min(octets, m0 + tile_tokens / 8);
   const T* xr = x + (size_t)row * n * kD + cb * 8;
@@ -157,7 +156,7 @@ __global__ void __launch_bounds__(kThreads) k_pack_octet_k(
         load8(xr + (size_t)i * kD, v);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          bytes |= (uint64_t)quant_code(v[e], af[e], inv[e], ad[e], bd[e], 1) << (8 * e + k);
+          bytes |= (uint64_t)code1(v[e], hi[e], lo[e]) << (8 * e + k);
       }
     }
     *reinterpret_cast<uint64_t*>(cr + (size_t)m * kD) = bytes;
@@ -174,6 +173,9 @@ __global__ void __launch_bounds__(kThreads) k_pack_octet_v(
   __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
   const int row = blockIdx.x;
   fold_stats<T>(part, row, S, 1, s_alpha, s_beta, s_inv, alpha_out, scale_out);
+  __shared__ float s_hi[kD], s_lo[kD];  // alpha + beta per channel as an exact pair
+  if (threadIdx.x < kD) two_sum(s_alpha[threadIdx.x], s_beta[threadIdx.x], s_hi[threadIdx.x], s_lo[threadIdx.x]);
+  __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int n_pad = (n + 255) / 256 * 256;
   const int b0 = blockIdx.y * (tile_tokens / 32), b1 = min(n_pad / 32, b0 + tile_tokens / 32);
@@ -182,16 +184,14 @@ __global__ void __launch_bounds__(kThreads) k_pack_octet_v(
   for (int blk = b0 + warp; blk < b1; blk += kThreads / 32) {
     const int i = blk * 32 + lane;
     uint32_t words[4] = {0, 0, 0, 0};  // channels lane, lane+32, lane+64, lane+96
-#pragma unroll 1
+#pragma unroll 4
     for (int cg = 0; cg < kD / 8; ++cg) {
       float v[8];
       if (i < n) load8(xr + (size_t)i * kD + cg * 8, v);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int j = cg * 8 + e;
-        const int code =
-            (i < n) ? quant_code(v[e], s_alpha[j], s_inv[j], (double)s_alpha[j], (double)s_beta[j], 1)
-                    : 0;
+        const uint32_t code = (i < n) ? code1(v[e], s_hi[j], s_lo[j]) : 0u;
         const uint32_t bal = __ballot_sync(0xffffffffu, code);
         if ((j & 31) == lane) words[j >> 5] = bal;
       }

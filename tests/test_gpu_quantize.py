@@ -125,3 +125,36 @@ def test_full_size_sampled_rows(cuda_device):
             _check_quantized(xr, sub, 1, layout)
     del q, k, v
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+def test_one_bit_midpoints_across_exponent_ranges(cuda_device, dtype):
+    """1-bit codes decide x > (alpha + beta) / 2 exactly even when alpha + beta
+    is not representable in float: channels span tiny to large magnitudes and
+    most tokens sit on or next to the exact midpoint."""
+    npd = np.float16 if dtype == "f16" else np.float32
+    rng = np.random.default_rng(11)
+    n, d = 96, 128
+    x = np.zeros((1, 1, n, d), dtype=npd)
+    for c in range(d):
+        lo_mag = float(npd(2.0 ** rng.integers(-14, 0)))
+        hi_mag = float(npd(rng.uniform(1.0, 6.0e4 if dtype == "f16" else 1.0e6)))
+        a, b = npd(-lo_mag if c % 2 else lo_mag), npd(hi_mag)
+        if a > b:
+            a, b = b, a
+        mid = (float(a) + float(b)) / 2.0  # exact in double
+        m = npd(mid)
+        around = [m]
+        for _ in range(6):
+            around.append(np.nextafter(around[-1], npd(np.inf), dtype=npd))
+        below = [m]
+        for _ in range(6):
+            below.append(np.nextafter(below[-1], npd(-np.inf), dtype=npd))
+        vals = [a, b] + around + below[1:]
+        col = np.array(vals + list(rng.uniform(float(a), float(b), n - len(vals))), dtype=npd)
+        x[0, 0, :, c] = col
+    xt = torch.from_numpy(x)
+    for layout in (cq.LAYOUT_CANONICAL, cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V):
+        qc = cq.cq_quantize_kv(xt.to(cuda_device), 1, layout)
+        torch.cuda.synchronize()
+        _check_quantized(xt, qc, 1, layout)
