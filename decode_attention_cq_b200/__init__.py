@@ -16,6 +16,8 @@ from .calibq import (  # noqa: F401
     QuantizedCache,
     cq_codes_bytes,
     cq_decode_attn,
+    cq_decode_attn_mixed,
+    cq_decode_attn_mixed_workspace_size,
     cq_decode_attn_workspace_size,
     cq_dequant,
     cq_quantize_kv,

@@ -31,6 +31,8 @@ ENTRY_POINTS = (
     "cq_quantize_kv_noalloc",
     "cq_decode_attn_workspace_size",
     "cq_decode_attn",
+    "cq_decode_attn_mixed_workspace_size",
+    "cq_decode_attn_mixed",
     "cq_dequant",
 )
 
@@ -56,6 +58,9 @@ _SIGS = {
     "cq_decode_attn_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "cq_decode_attn": ([_P, _I, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F,
                         cq_calib, _P, _P, _SZ, _P], _I),
+    "cq_decode_attn_mixed_workspace_size": ([_I, _I, _I, ctypes.POINTER(_SZ)], _I),
+    "cq_decode_attn_mixed": ([_P, _I, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _I, _I, _I, _I, _I, _F,
+                              cq_calib, _P, _P, _SZ, _P], _I),
     "cq_dequant": ([_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P], _I),
 }
 
@@ -203,6 +208,37 @@ def cq_decode_attn(q: torch.Tensor, k: QuantizedCache, v: QuantizedCache, *,
                                  B, Hq, Hkv, n, d, k.bits, float(softmax_scale), cal, _ptr(out),
                                  _ptr(workspace), 0 if workspace is None else workspace.numel(),
                                  _stream(stream)), "cq_decode_attn")
+    return out
+
+
+def cq_decode_attn_mixed_workspace_size(B: int, Hq: int, d: int) -> int:
+    out = ctypes.c_size_t()
+    _check(load().cq_decode_attn_mixed_workspace_size(B, Hq, d, ctypes.byref(out)),
+           "cq_decode_attn_mixed_workspace_size")
+    return out.value
+
+
+def cq_decode_attn_mixed(q: torch.Tensor, k: QuantizedCache, v: QuantizedCache,
+                         k_text: torch.Tensor | None, v_text: torch.Tensor | None, *,
+                         calib=(False, 1.0, 1.0), softmax_scale: float = 0.0,
+                         out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """Decode over quantized visual K/V (octet layouts) followed by full-precision
+    text K/V [B, Hkv, n_text, d] in q's dtype (None or n_text = 0 for none)."""
+    B, Hq, d = q.shape
+    _, Hkv, n, _ = k.shape
+    n_text = 0 if k_text is None else k_text.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = torch.empty(cq_decode_attn_mixed_workspace_size(B, Hq, d), dtype=torch.uint8,
+                                device=q.device)
+    cal = cq_calib(int(bool(calib[0])), float(calib[1]), float(calib[2]))
+    _check(load().cq_decode_attn_mixed(_ptr(q), _dt(q), _ptr(k.codes), _ptr(k.alpha), _ptr(k.scale),
+                                       _ptr(v.codes), _ptr(v.alpha), _ptr(v.scale), n, k.bits,
+                                       _ptr(k_text), _ptr(v_text), n_text, B, Hq, Hkv, d,
+                                       float(softmax_scale), cal, _ptr(out), _ptr(workspace),
+                                       workspace.numel(), _stream(stream)), "cq_decode_attn_mixed")
     return out
 
 

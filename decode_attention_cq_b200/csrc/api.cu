@@ -81,6 +81,30 @@ cq_status row_bytes(cq_layout layout, int n, int bits, size_t* out) {
 
 cq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CQ_OK : CQ_ERR_CUDA; }
 
+cq::DecodeArgs make_args(const void* q, const uint8_t* k_codes, const void* k_alpha, const void* k_scale,
+                         const uint8_t* v_codes, const void* v_alpha, const void* v_scale, int B, int Hq, int Hkv,
+                         int n, int d, int bits, float softmax_scale, cq_calib calib, void* out) {
+  cq::DecodeArgs a;
+  a.q = q;
+  a.k_codes = k_codes;
+  a.k_alpha = k_alpha;
+  a.k_scale = k_scale;
+  a.v_codes = v_codes;
+  a.v_alpha = v_alpha;
+  a.v_scale = v_scale;
+  a.out = out;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.n = n;
+  a.bits = bits;
+  a.sigma = softmax_scale == 0.f ? 1.0f / sqrtf((float)d) : softmax_scale;
+  a.calib = calib.enabled ? 1 : 0;
+  a.tau_lo = calib.tau_lo;
+  a.tau_hi = calib.tau_hi;
+  return a;
+}
+
 }  // namespace
 
 extern "C" {
@@ -192,24 +216,8 @@ cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, con
     return CQ_ERR_UNSUPPORTED;
   const void* ptrs[] = {q, k_codes, k_alpha, k_scale, v_codes, v_alpha, v_scale, out};
   for (const void* p : ptrs) CQ_TRY(check_ptr(p));
-  cq::DecodeArgs a;
-  a.q = q;
-  a.k_codes = k_codes;
-  a.k_alpha = k_alpha;
-  a.k_scale = k_scale;
-  a.v_codes = v_codes;
-  a.v_alpha = v_alpha;
-  a.v_scale = v_scale;
-  a.out = out;
-  a.B = B;
-  a.Hq = Hq;
-  a.Hkv = Hkv;
-  a.n = n;
-  a.bits = bits;
-  a.sigma = softmax_scale == 0.f ? 1.0f / sqrtf((float)d) : softmax_scale;
-  a.calib = calib.enabled ? 1 : 0;
-  a.tau_lo = calib.tau_lo;
-  a.tau_hi = calib.tau_hi;
+  cq::DecodeArgs a = make_args(q, k_codes, k_alpha, k_scale, v_codes, v_alpha, v_scale, B, Hq, Hkv, n, d, bits,
+                               softmax_scale, calib, out);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (generic) {
     const size_t need = cq::decode_generic_workspace_bytes(B, Hq, n);
@@ -222,6 +230,47 @@ cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, con
                                                                             : cq::launch_decode_octet(a, dt, s);
   if (e == cudaErrorNotSupported) return CQ_ERR_UNSUPPORTED;
   return cuda_status(e);
+}
+
+cq_status cq_decode_attn_mixed_workspace_size(int B, int Hq, int d, size_t* bytes) {
+  if (bytes == nullptr || B < 1 || Hq < 1) return CQ_ERR_INVALID_ARG;
+  if (d != kD) return CQ_ERR_UNSUPPORTED;
+  *bytes = cq::text_merge_workspace_bytes(B, Hq);
+  return CQ_OK;
+}
+
+cq_status cq_decode_attn_mixed(const void* q, cq_dtype dt, const uint8_t* k_codes, const void* k_alpha,
+                               const void* k_scale, const uint8_t* v_codes, const void* v_alpha,
+                               const void* v_scale, int n_vis, int bits, const void* k_text, const void* v_text,
+                               int n_text, int B, int Hq, int Hkv, int d, float softmax_scale, cq_calib calib,
+                               void* out, void* workspace, size_t ws_bytes, cq_stream_t stream) {
+  if (!valid_dtype(dt)) return CQ_ERR_INVALID_ARG;
+  CQ_TRY(check_shape(B, Hq, n_vis, d, bits));
+  if (Hkv < 1 || Hq % Hkv || n_text < 0) return CQ_ERR_INVALID_ARG;
+  if (!isfinite(softmax_scale) || softmax_scale < 0.f) return CQ_ERR_INVALID_ARG;
+  if (calib.enabled && (!isfinite(calib.tau_lo) || !isfinite(calib.tau_hi))) return CQ_ERR_INVALID_ARG;
+  if ((double)B * Hkv * n_text * d > 9.0e15) return CQ_ERR_INVALID_ARG;
+  if (Hq / Hkv != 4) return CQ_ERR_UNSUPPORTED;
+  if (bits == 1 ? !cq::decode_mma_supports(n_vis) : !cq::decode_ring_supports(n_vis, bits))
+    return CQ_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k_codes, k_alpha, k_scale, v_codes, v_alpha, v_scale, out};
+  for (const void* p : ptrs) CQ_TRY(check_ptr(p));
+  if (n_text > 0) {
+    CQ_TRY(check_ptr(k_text));
+    CQ_TRY(check_ptr(v_text));
+  }
+  const size_t need = cq::text_merge_workspace_bytes(B, Hq);
+  if (workspace == nullptr || ws_bytes < need) return CQ_ERR_WORKSPACE;
+  CQ_TRY(check_ptr(workspace));
+  cq::DecodeArgs a = make_args(q, k_codes, k_alpha, k_scale, v_codes, v_alpha, v_scale, B, Hq, Hkv, n_vis, d,
+                               bits, softmax_scale, calib, out);
+  a.part_o = static_cast<float*>(workspace);
+  a.part_lse = a.part_o + (size_t)B * Hq * kD;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = bits != 1 ? cq::launch_decode_ring(a, dt, s) : cq::launch_decode_mma(a, dt, s);
+  if (e == cudaErrorNotSupported) return CQ_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return CQ_ERR_CUDA;
+  return cuda_status(cq::launch_text_merge(a, dt, k_text, v_text, n_text, s));
 }
 
 cq_status cq_dequant(const uint8_t* codes, const void* alpha, const void* scale, cq_dtype dt,

@@ -59,6 +59,7 @@ struct RingFixed {
   float part_l[kMaxCl][kG];         // every peer's sum of weights (pushed to all)
   float lsum[kWarps][kG];           // per-warp sum of weights
   float c0[kG], kscale[kG], alog2[kG], ref[kG];
+  float cst[kG];                    // g(x) - slope x: the calibration's constant term
   float recv[kRecv];                // [src][h][channel - first owned channel]
 };
 
@@ -298,10 +299,14 @@ __global__ void __launch_bounds__(kThreads, ring_slots<BITS>() == 2 ? 3 : 2)
       m = fminf(m, F.mM[r][t][0]);
       M = fmaxf(M, F.mM[r][t][1]);
     }
-    float slope = 1.f;
-    if (a.calib && M > m) slope = (a.tau_hi * M - a.tau_lo * m) / (M - m);
+    float slope = 1.f, cst = 0.f;
+    if (a.calib && M > m) {
+      slope = (a.tau_hi * M - a.tau_lo * m) / (M - m);
+      cst = a.tau_lo * m - slope * m;  // g(x) = slope x + cst
+    }
     F.alog2[t] = slope * kLog2e;
     F.ref[t] = fmaxf(slope * m, slope * M) * kLog2e;
+    F.cst[t] = cst;
   }
   __syncthreads();
 
@@ -461,8 +466,14 @@ __global__ void __launch_bounds__(kThreads, ring_slots<BITS>() == 2 ? 3 : 2)
       }
       const float alpha = DT<T>::f(sRows[6 * kD + ch]);
       const float step = *err ? __int_as_float(0x7fc00000) : DT<T>::f(sRows[7 * kD + ch]);
-      T* out = static_cast<T*>(a.out) + ((size_t)b * a.Hq + (size_t)kG * hkv + h) * kD;
-      out[ch] = DT<T>::from_float(fmaf(step, s / l, alpha));
+      const size_t bh = (size_t)b * a.Hq + (size_t)kG * hkv + h;
+      if (a.part_o == nullptr) {
+        static_cast<T*>(a.out)[bh * kD + ch] = DT<T>::from_float(fmaf(step, s / l, alpha));
+      } else {
+        a.part_o[bh * kD + ch] = fmaf(step, s / l, alpha);
+        // sum_i exp(y_i) = 2^ref sum_i p_i e^cst with p_i = 2^(x_i alog2 - ref)
+        if (ch == 0) a.part_lse[bh] = fmaf(F.ref[h], 0.6931471805599453f, logf(l)) + F.cst[h];
+      }
     }
   }
   if (*err && t == 0) {  // let copies still in flight land before the CTA's memory is reused

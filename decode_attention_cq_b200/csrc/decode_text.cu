@@ -1,0 +1,137 @@
+// Mixed caches: the full-precision text tokens next to a quantized visual
+// cache (the CalibQuant article quantizes the visual KV cache; text tokens keep
+// their precision). The visual part is attended by an octet decode kernel in
+// partial mode (normalized fp32 result + ln sum exp of its calibrated logits);
+// this kernel attends the G = 4 query heads of one (batch, kv-head) row over
+// the text keys / values with an online softmax on the raw logits sigma q.k,
+// and merges both parts by their log-sum-exps into the final output:
+//   o = (e^{lse_v} o_v + sum_j e^{x_j} v_j) / (e^{lse_v} + sum_j e^{x_j}).
+#include <float.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace cq {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kG = 4;
+
+// Four consecutive elements of a row as floats.
+__device__ __forceinline__ void load4(const half* p, float (&v)[4]) {
+  const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+  const float2 a = __half22float2(*reinterpret_cast<const half2*>(&u.x));
+  const float2 b = __half22float2(*reinterpret_cast<const half2*>(&u.y));
+  v[0] = a.x;
+  v[1] = a.y;
+  v[2] = b.x;
+  v[3] = b.y;
+}
+__device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  v[0] = a.x;
+  v[1] = a.y;
+  v[2] = a.z;
+  v[3] = a.w;
+}
+
+// grid: one CTA per (batch, kv-head) row; warp w takes text tokens w, w + 8, ...;
+// lane l holds channels 4 l .. 4 l + 3.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_text_merge(const T* __restrict__ q, const T* __restrict__ kt,
+                                                         const T* __restrict__ vt, int n_text,
+                                                         const float* __restrict__ part_o,
+                                                         const float* __restrict__ part_lse, T* __restrict__ out,
+                                                         int Hq, int Hkv, float sigma) {
+  __shared__ float s_m[kWarps][kG], s_l[kWarps][kG];
+  __shared__ float s_acc[kWarps][kG][kD];
+  const int row = blockIdx.x, b = row / Hkv, hkv = row % Hkv;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const size_t bh0 = (size_t)b * Hq + (size_t)kG * hkv;  // first query head of the row
+
+  float qv[kG][4];
+#pragma unroll
+  for (int h = 0; h < kG; ++h) load4(q + (bh0 + h) * kD + 4 * lane, qv[h]);
+  float m[kG], l[kG], acc[kG][4];
+#pragma unroll
+  for (int h = 0; h < kG; ++h) {
+    m[h] = -FLT_MAX;
+    l[h] = 0.f;
+    acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
+  }
+  const T* kr = kt + (size_t)row * n_text * kD + 4 * lane;
+  const T* vr = vt + (size_t)row * n_text * kD + 4 * lane;
+  for (int j = warp; j < n_text; j += kWarps) {
+    float kv[4], vv[4];
+    load4(kr + (size_t)j * kD, kv);
+    load4(vr + (size_t)j * kD, vv);
+#pragma unroll
+    for (int h = 0; h < kG; ++h) {
+      float dot = qv[h][0] * kv[0] + qv[h][1] * kv[1] + qv[h][2] * kv[2] + qv[h][3] * kv[3];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      const float x = sigma * dot;
+      const float mn = fmaxf(m[h], x);
+      const float sc = expf(m[h] - mn), p = expf(x - mn);
+      l[h] = fmaf(l[h], sc, p);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[h][c] = fmaf(acc[h][c], sc, p * vv[c]);
+      m[h] = mn;
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < kG; ++h) {
+    if (lane == 0) {
+      s_m[warp][h] = m[h];
+      s_l[warp][h] = l[h];
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) s_acc[warp][h][4 * lane + c] = acc[h][c];
+  }
+  __syncthreads();
+  // thread (h, ch), two per thread: merge the warps' text parts and the visual part
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int idx = 2 * t + e, h = idx >> 7, ch = idx & 127;
+    const size_t bh = bh0 + h;
+    const float lse_v = part_lse[bh];
+    float M = lse_v;
+    for (int w = 0; w < kWarps; ++w)
+      if (s_l[w][h] > 0.f) M = fmaxf(M, s_m[w][h]);
+    const float wv = expf(lse_v - M);
+    float num = wv * part_o[bh * kD + ch], den = wv;
+    for (int w = 0; w < kWarps; ++w) {
+      if (s_l[w][h] > 0.f) {
+        const float f = expf(s_m[w][h] - M);
+        num = fmaf(f, s_acc[w][h][ch], num);
+        den = fmaf(f, s_l[w][h], den);
+      }
+    }
+    out[bh * kD + ch] = DT<T>::from_float(num / den);
+  }
+}
+
+}  // namespace
+
+size_t text_merge_workspace_bytes(int B, int Hq) {
+  return (size_t)B * Hq * kD * sizeof(float) + (size_t)B * Hq * sizeof(float);
+}
+
+cudaError_t launch_text_merge(const DecodeArgs& a, cq_dtype dt, const void* k_text, const void* v_text, int n_text,
+                              cudaStream_t stream) {
+  const int rows = a.B * a.Hkv;
+  if (dt == CQ_F16)
+    k_text_merge<half><<<rows, kThreads, 0, stream>>>(
+        static_cast<const half*>(a.q), static_cast<const half*>(k_text), static_cast<const half*>(v_text), n_text,
+        a.part_o, a.part_lse, static_cast<half*>(a.out), a.Hq, a.Hkv, a.sigma);
+  else
+    k_text_merge<float><<<rows, kThreads, 0, stream>>>(
+        static_cast<const float*>(a.q), static_cast<const float*>(k_text), static_cast<const float*>(v_text), n_text,
+        a.part_o, a.part_lse, static_cast<float*>(a.out), a.Hq, a.Hkv, a.sigma);
+  return cudaGetLastError();
+}
+
+}  // namespace cq

@@ -40,6 +40,11 @@ struct DecodeArgs {
   float sigma;
   int calib;
   float tau_lo, tau_hi;
+  // Partial mode (octet kernels only): when part_o is set, the kernel writes the
+  // normalized result in fp32 to part_o [B][Hq][d] and ln sum_i exp(y_i) of the
+  // calibrated logits y = g(x) to part_lse [B][Hq] instead of writing out.
+  float* part_o = nullptr;
+  float* part_lse = nullptr;
 };
 size_t decode_generic_workspace_bytes(int B, int Hq, int n);
 cudaError_t launch_decode_generic(const DecodeArgs& a, cq_dtype dt, void* workspace,
@@ -47,6 +52,12 @@ cudaError_t launch_decode_generic(const DecodeArgs& a, cq_dtype dt, void* worksp
 
 // ---- decode_octet.cu (octet layouts, bits = 1, Hq = 4 Hkv, tensor cores)
 cudaError_t launch_decode_octet(const DecodeArgs& a, cq_dtype dt, cudaStream_t stream);
+
+// ---- decode_text.cu (mixed caches: full-precision text tokens + merge with the
+// partial result of a quantized visual part; G = 4)
+size_t text_merge_workspace_bytes(int B, int Hq);
+cudaError_t launch_text_merge(const DecodeArgs& a, cq_dtype dt, const void* k_text, const void* v_text, int n_text,
+                              cudaStream_t stream);
 
 // ---- decode_ring.cu (octet layouts, bits in {2, 4, 8}, Hq = 4 Hkv, n <= 32768, mma.sync)
 bool decode_ring_supports(int n, int bits);

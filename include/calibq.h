@@ -207,6 +207,41 @@ cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, con
                          cq_stream_t stream);
 
 /*
+ * Workspace of cq_decode_attn_mixed: the visual part's partial result
+ * (B * Hq * d floats) and its log-sum-exps (B * Hq floats).
+ */
+cq_status cq_decode_attn_mixed_workspace_size(int B, int Hq, int d, size_t* bytes);
+
+/*
+ * One decode step over a mixed cache: n_vis quantized visual tokens (the
+ * article quantizes the visual KV cache) followed by n_text full-precision
+ * text tokens, in one softmax:
+ *
+ *   x_i = sigma * ( q . alpha_K + (q (.) s_K) . c^K_i )   visual logits (Method 2)
+ *   y_i = g(x_i), g fitted to the range of the visual logits only (Method 3)
+ *   z_j = sigma * q . k_j                                 text logits, not calibrated
+ *   o   = ( sum_i e^{y_i} (alpha_V + s_V (.) c^V_i) + sum_j e^{z_j} v_j )
+ *         / ( sum_i e^{y_i} + sum_j e^{z_j} )
+ *
+ * (Which tokens the calibration sees, and that g's constant term is kept so
+ * that visual and text logits share one scale, is this library's reading; the
+ * article applies g to the scores of the quantized cache.)
+ *
+ *   visual codes: k_codes in CQ_LAYOUT_OCTET_K, v_codes in CQ_LAYOUT_OCTET_V,
+ *     bits in {1, 2, 4, 8}, statistics [B][Hkv][d] in `dt`;
+ *   k_text, v_text: [B][Hkv][n_text][d] in `dt` (may be NULL when n_text = 0);
+ *   q, out: [B][Hq][d] in `dt`; Hq = 4 * Hkv; d = 128;
+ *   n_vis <= 32768; workspace: cq_decode_attn_mixed_workspace_size bytes.
+ * Two launches on `stream` (visual partial, then text + merge).
+ */
+cq_status cq_decode_attn_mixed(const void* q, cq_dtype dt, const uint8_t* k_codes, const void* k_alpha,
+                               const void* k_scale, const uint8_t* v_codes, const void* v_alpha,
+                               const void* v_scale, int n_vis, int bits, const void* k_text,
+                               const void* v_text, int n_text, int B, int Hq, int Hkv, int d,
+                               float softmax_scale, cq_calib calib, void* out, void* workspace,
+                               size_t ws_bytes, cq_stream_t stream);
+
+/*
  * Dequantize packed codes back to floating point (for checks only):
  *   out[b][h][i][j] = alpha[b][h][j] + scale[b][h][j] * code(i, j),
  * evaluated in double and rounded once to `dt`.

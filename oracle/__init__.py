@@ -20,8 +20,7 @@ Citations name the CalibQuant article (QbitAI's Chinese write-up of
 * "Runtime analysis" -- the decode-throughput measurement.
 
 The formulas of that page were lost when it was converted to text; where a step
-is open, the reading taken is stated in the function's docstring and collected
-in DESIGN.md.
+is open, the reading taken is stated in the function's docstring.
 
 Parity status: every public function here is pinned by ``tests/test_oracle_*``
 against closed forms, exact rational arithmetic on small inputs, a library
@@ -42,6 +41,7 @@ from .calibquant import (  # noqa: F401
     attend_post_scaled,
     quantize_cache,
     decode_attention,
+    decode_attention_mixed,
 )
 from .layouts import (  # noqa: F401
     LAYOUT_CANONICAL,

@@ -29,6 +29,7 @@ __all__ = [
     "attend_post_scaled",
     "quantize_cache",
     "decode_attention",
+    "decode_attention_mixed",
 ]
 
 _STORE = {"f16": np.float16, "f32": np.float32}
@@ -257,3 +258,33 @@ def decode_attention(q, k, v, bits: int, dtype: str, calib=(False, 1.0, 1.0),
         vmag = attend_dequantized(p, np.abs(v_hat))
         assert np.all(np.abs(out - o2) <= 1e-12 * (vmag + 1e-300)), "post-scaled output disagrees"
     return {"out": out, "scores": x, "y": y, "p": p, "kq": kq, "vq": vq}
+
+
+def decode_attention_mixed(q, k_vis, v_vis, k_text, v_text, bits: int, dtype: str,
+                           calib=(False, 1.0, 1.0), softmax_scale: float = 0.0):
+    """One decode step over a mixed cache: quantized visual tokens, then
+    full-precision text tokens, in one softmax, in float64.
+
+    The article quantizes the visual KV cache (Methods 1 and 2) and calibrates
+    the scores of that quantized cache (Method 3). Reading for a cache that also
+    holds text tokens: g is fitted to the range of the visual logits only and
+    applied to them with its constant term (so visual and text logits share one
+    scale); text logits sigma <q, k_j> are used as they are and their values
+    as stored.
+
+    q: ``[B, Hq, d]``; k_vis, v_vis: ``[B, Hkv, n_vis, d]`` (full precision,
+    quantized here); k_text, v_text: ``[B, Hkv, n_text, d]``.
+    Returns dict(out [B, Hq, d], p [B, Hq, n_vis + n_text]).
+    """
+    enabled, tau_lo, tau_hi = calib
+    kq = quantize_cache(k_vis, bits, dtype)
+    vq = quantize_cache(v_vis, bits, dtype)
+    k_hat = dequantize(kq["codes"], kq["alpha"], kq["scale"])
+    v_hat = dequantize(vq["codes"], vq["alpha"], vq["scale"])
+    x = scores_dequantized(q, k_hat, softmax_scale)
+    y = calibrate(x, tau_lo, tau_hi) if enabled else x
+    z = scores_dequantized(q, k_text, softmax_scale)  # plain sigma <q, k_j>
+    p = softmax(np.concatenate([y, z], axis=-1))
+    n_vis = y.shape[-1]
+    out = attend_dequantized(p[..., :n_vis], v_hat) + attend_dequantized(p[..., n_vis:], _f64(v_text))
+    return {"out": out, "p": p}

@@ -299,3 +299,63 @@ def test_eight_bits_approach_exact_attention():
     bound = (np.exp(2 * eps)[..., None] - 1) * vrange + sv
     assert np.all(np.abs(r["out"] - exact) <= bound)
     assert np.max(np.abs(r["out"] - exact)) < 0.05 * np.max(np.abs(exact))
+
+
+def _text(seed, B, Hkv, n_text, d):
+    g = torch.Generator().manual_seed(seed)
+    return (synth.make_cache(B, Hkv, n_text, d, "f16", 0, g, "cpu").to(torch.float64).numpy(),
+            synth.make_cache(B, Hkv, n_text, d, "f16", 0, g, "cpu").to(torch.float64).numpy())
+
+
+def test_mixed_cache_without_text_is_plain_decode():
+    q, k, v = _case(seed=71)
+    kt = np.zeros((k.shape[0], k.shape[1], 0, k.shape[3]))
+    for calib in ((False, 1, 1), (True, 0.8, 0.9)):
+        r = oracle.decode_attention(q, k, v, 1, "f16", calib)
+        rm = oracle.decode_attention_mixed(q, k, v, kt, kt, 1, "f16", calib)
+        assert np.allclose(rm["out"], r["out"], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("bits", [1, 4])
+def test_mixed_cache_matches_library_sdpa(bits):
+    """Uncalibrated: textbook attention over [dequantized visual; text] tokens.
+    Calibrated: the visual logits become a x + c (a = slope, c = the constant of
+    the map [m, M] -> [tau_lo m, tau_hi M]), i.e. keys scaled by a and an additive
+    mask c on the visual positions."""
+    q, k, v = _case(seed=73, B=1, Hq=4, Hkv=1)
+    kt, vt = _text(74, 1, 1, 17, q.shape[-1])
+    r0 = oracle.decode_attention(q, k, v, bits, "f16", (False, 1, 1))
+    kh = oracle.dequantize(r0["kq"]["codes"], r0["kq"]["alpha"], r0["kq"]["scale"])
+    vh = oracle.dequantize(r0["vq"]["codes"], r0["vq"]["alpha"], r0["vq"]["scale"])
+    d, n_vis = q.shape[-1], k.shape[2]
+    sig = 1 / np.sqrt(d)
+    rm = oracle.decode_attention_mixed(q, k, v, kt, vt, bits, "f16", (False, 1, 1))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[:, :, None, :], torch.from_numpy(np.repeat(np.concatenate([kh, kt], 2), 4, 1)),
+        torch.from_numpy(np.repeat(np.concatenate([vh, vt], 2), 4, 1)))[:, :, 0].numpy()
+    assert np.allclose(rm["out"], ref, rtol=1e-10, atol=1e-10)
+    tau = (0.8, 0.9)
+    rc = oracle.decode_attention_mixed(q, k, v, kt, vt, bits, "f16", (True, *tau))
+    x = sig * np.einsum("bhd,bnd->bhn", q, kh[:, 0])  # visual logits, every head
+    m, M = x.min(-1), x.max(-1)
+    a = (tau[1] * M - tau[0] * m) / (M - m)
+    c = tau[0] * m - a * m
+    for h in range(4):
+        keys = np.concatenate([a[0, h] * kh[0, 0], kt[0, 0]], 0)[None, None]
+        vals = np.concatenate([vh[0, 0], vt[0, 0]], 0)[None, None]
+        mask = np.concatenate([np.full(n_vis, c[0, h]), np.zeros(kt.shape[2])])[None, None, None, :]
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[:, h:h + 1])[:, :, None, :], torch.from_numpy(keys), torch.from_numpy(vals),
+            attn_mask=torch.from_numpy(mask))
+        assert np.allclose(rc["out"][0, h], ref[0, 0, 0].numpy(), rtol=1e-10, atol=1e-10)
+
+
+def test_mixed_cache_duplicate_tokens_leave_attention_unchanged():
+    """Text tokens equal to the dequantized visual tokens (calibration off):
+    every token appears twice, which does not change the softmax average."""
+    q, k, v = _case(seed=75)
+    r = oracle.decode_attention(q, k, v, 2, "f16", (False, 1, 1))
+    kh = oracle.dequantize(r["kq"]["codes"], r["kq"]["alpha"], r["kq"]["scale"])
+    vh = oracle.dequantize(r["vq"]["codes"], r["vq"]["alpha"], r["vq"]["scale"])
+    rm = oracle.decode_attention_mixed(q, k, v, kh, vh, 2, "f16", (False, 1, 1))
+    assert np.allclose(rm["out"], r["out"], rtol=1e-12, atol=1e-12)
