@@ -197,12 +197,29 @@ def run_ours(args, world, rank, local):
     torch.cuda.empty_cache()
 
     out = torch.empty_like(q)
-    dws_n = cq.cq_decode_attn_workspace_size(layouts[0], layouts[1], B, w.hq, w.hkv, n, w.d, bits)
-    dws = torch.empty(dws_n, dtype=torch.uint8, device=device) if dws_n else None
-    launches_per_step = 1 if args.path == "octet" else 3
+    n_text = args.text
+    if n_text:  # mixed cache: full-precision text tokens after the quantized visual ones
+        if args.path != "octet":
+            raise SystemExit("--text needs the octet layouts")
+        gt = torch.Generator(device=device)
+        gt.manual_seed(w.seed + 7 + 1000 * rank)
+        k_text = synth.make_cache(B, w.hkv, n_text, w.d, w.dtype, 0, gt, device)
+        v_text = synth.make_cache(B, w.hkv, n_text, w.d, w.dtype, 0, gt, device)
+        dws = torch.empty(cq.cq_decode_attn_mixed_workspace_size(B, w.hq, w.d), dtype=torch.uint8, device=device)
+        launches_per_step = 2
+    else:
+        dws_n = cq.cq_decode_attn_workspace_size(layouts[0], layouts[1], B, w.hq, w.hkv, n, w.d, bits)
+        dws = torch.empty(dws_n, dtype=torch.uint8, device=device) if dws_n else None
+        launches_per_step = 1 if args.path == "octet" else 3
+
+    def decode(qq):
+        if n_text:
+            cq.cq_decode_attn_mixed(qq, kq, vq, k_text, v_text, calib=CALIB, out=out, workspace=dws)
+        else:
+            cq.cq_decode_attn(qq, kq, vq, calib=CALIB, out=out, workspace=dws)
 
     def step():
-        cq.cq_decode_attn(q, kq, vq, calib=CALIB, out=out, workspace=dws)
+        decode(q)
 
     for it in range(args.warmup):
         flush.fill_(it & 255)
@@ -267,7 +284,7 @@ def run_ours(args, world, rank, local):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         q_dev.copy_(q_host, non_blocking=True)
-        cq.cq_decode_attn(q_dev, kq, vq, calib=CALIB, out=out, workspace=dws)
+        decode(q_dev)
         out_host.copy_(out, non_blocking=True)
         e1.record(stream)
         e1.synchronize()
@@ -276,10 +293,11 @@ def run_ours(args, world, rank, local):
     e2e_mean = max_over_ranks(sum(e2e_ms) / len(e2e_ms), world, device)
 
     peak, peak_src = measured_peaks()
-    alg = algorithmic_bytes(B, w.hq, w.hkv, n, w.d, bits)
-    kernel_ms = sum(step_ms) / len(step_ms)  # one launch per step on the octet path
+    dsize = 2 if w.dtype == "f16" else 4
+    alg = algorithmic_bytes(B, w.hq, w.hkv, n, w.d, bits, dsize) + 2 * B * w.hkv * n_text * w.d * dsize
+    kernel_ms = sum(step_ms) / len(step_ms)  # the step's launches (one on the plain octet path)
     achieved = alg / (kernel_ms * 1e-3) / 1e9
-    trec = traffic_record(args.path, args.workload, bits)
+    trec = None if n_text else traffic_record(args.path, args.workload, bits)
     fill_mean = sum(fill_ms) / len(fill_ms)
     fill_alg = cache_fill_bytes(B, w.hkv, n, w.d, bits)
     line = {
@@ -298,14 +316,17 @@ def run_ours(args, world, rank, local):
         "data": "synthetic (seeded InternVL-2.5-shaped K/V caches, no dataset or checkpoint)",
         "config": {"workload": args.workload, "batch_per_gpu": B, "global_batch": B * world,
                    "q_heads": w.hq, "kv_heads": w.hkv, "head_dim": w.d, "n_tokens": n, "bits": bits,
-                   "layout": args.path, "calibration": {"tau_lo": CALIB[1], "tau_hi": CALIB[2]},
+                   "layout": args.path, "text_tokens": n_text,
+                   "calibration": {"tau_lo": CALIB[1], "tau_hi": CALIB[2]},
                    "l2": "flushed (256 MB write) between timed steps",
                    "parallelism": f"dp{world} (independent sequences per GPU)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_src,
                      "traffic": None if trec is None else trec["dram_bytes_per_launch"],
                      "algorithmic_bytes_per_launch": alg,
-                     "kernel": "k_decode_mma" if args.path == "octet" else "k_scores + k_softmax_v + k_merge"},
+                     "kernel": ("k_scores + k_softmax_v + k_merge" if args.path != "octet"
+                                else ("k_decode_mma" if bits == 1 else f"k_decode_ring<{bits}>")
+                                + (" (partial) + k_text_merge" if n_text else ""))},
         "cache_fill": {"ms": fill_mean, "algorithmic_bytes": fill_alg,
                        "achieved_gbs": fill_alg / (fill_mean * 1e-3) / 1e9},
         "e2e": {"value": total_tokens / (e2e_mean * 1e-3), "unit": "tokens/s",
@@ -395,6 +416,8 @@ def main():
     ap.add_argument("--batch", type=int, default=0)
     ap.add_argument("--bits", type=int, default=1)
     ap.add_argument("--path", choices=["octet", "canonical"], default="octet")
+    ap.add_argument("--text", type=int, default=0,
+                    help="full-precision text tokens after the quantized ones (mixed cache)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args_global = args

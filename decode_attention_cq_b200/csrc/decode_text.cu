@@ -38,18 +38,23 @@ __device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
   v[3] = a.w;
 }
 
-// grid: one CTA per (batch, kv-head) row; warp w takes text tokens w, w + 8, ...;
-// lane l holds channels 4 l .. 4 l + 3.
+// grid: one CTA per (batch, kv-head) row. Warp w takes batches of 8 text
+// tokens (batch w, w + 8, ...); lane l holds channels 4 l .. 4 l + 3 of the
+// keys and values. The 32 partial dot products of a batch (8 tokens x 4 heads)
+// are summed over the lanes with one transposed butterfly (31 shuffles), after
+// which lane l owns the logit of token l / 4, head l % 4.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_text_merge(const T* __restrict__ q, const T* __restrict__ kt,
                                                          const T* __restrict__ vt, int n_text,
                                                          const float* __restrict__ part_o,
                                                          const float* __restrict__ part_lse, T* __restrict__ out,
                                                          int Hq, int Hkv, float sigma) {
+  constexpr int kBatch = 8;
   __shared__ float s_m[kWarps][kG], s_l[kWarps][kG];
   __shared__ float s_acc[kWarps][kG][kD];
   const int row = blockIdx.x, b = row / Hkv, hkv = row % Hkv;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int my_h = lane & 3;  // head of the logit this lane owns after the butterfly
   const size_t bh0 = (size_t)b * Hq + (size_t)kG * hkv;  // first query head of the row
 
   float qv[kG][4];
@@ -64,22 +69,68 @@ __global__ void __launch_bounds__(kThreads) k_text_merge(const T* __restrict__ q
   }
   const T* kr = kt + (size_t)row * n_text * kD + 4 * lane;
   const T* vr = vt + (size_t)row * n_text * kD + 4 * lane;
-  for (int j = warp; j < n_text; j += kWarps) {
-    float kv[4], vv[4];
-    load4(kr + (size_t)j * kD, kv);
-    load4(vr + (size_t)j * kD, vv);
+  for (int j0 = kBatch * warp; j0 < n_text; j0 += kBatch * kWarps) {
+    float dv[kBatch * kG];  // partial dots, index 4 token + head
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      float kv[4] = {0.f, 0.f, 0.f, 0.f};
+      if (j0 + u < n_text) load4(kr + (size_t)(j0 + u) * kD, kv);
+#pragma unroll
+      for (int h = 0; h < kG; ++h)
+        dv[kG * u + h] = qv[h][0] * kv[0] + qv[h][1] * kv[1] + qv[h][2] * kv[2] + qv[h][3] * kv[3];
+    }
+    // transposed butterfly: after the step with offset s, lane l keeps the
+    // indices whose bit s matches its own; at the end dv[0] = full dot of index l
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) {
+      const bool upper = lane & s;
+#pragma unroll
+      for (int i = 0; i < s; ++i) {
+        const float send = upper ? dv[i] : dv[i + s];
+        const float keep = upper ? dv[i + s] : dv[i];
+        dv[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+      }
+    }
+    const bool valid = j0 + (lane >> 2) < n_text;
+    const float x = valid ? sigma * dv[0] : -FLT_MAX;
+    // batch maximum and weights per head: lanes with equal lane % 4
+    float bm = x;
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+    float mine_m = m[0];
+#pragma unroll
+    for (int h = 1; h < kG; ++h)
+      if (my_h == h) mine_m = m[h];
+    const float mn = fmaxf(mine_m, bm);
+    const float p = valid ? expf(x - mn) : 0.f;
+    const float sc = expf(mine_m - mn);
+    float ps = p;
+    ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+    ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+    ps += __shfl_xor_sync(0xffffffffu, ps, 16);
+    // every lane updates its 4 channels of all 4 heads
+    float vv[kBatch][4];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      vv[u][0] = vv[u][1] = vv[u][2] = vv[u][3] = 0.f;
+      if (j0 + u < n_text) load4(vr + (size_t)(j0 + u) * kD, vv[u]);
+    }
 #pragma unroll
     for (int h = 0; h < kG; ++h) {
-      float dot = qv[h][0] * kv[0] + qv[h][1] * kv[1] + qv[h][2] * kv[2] + qv[h][3] * kv[3];
+      const float sch = __shfl_sync(0xffffffffu, sc, h);
+      const float mh = __shfl_sync(0xffffffffu, mn, h);
+      const float lh = __shfl_sync(0xffffffffu, ps, h);
+      l[h] = fmaf(l[h], sch, lh);
+      m[h] = mh;
 #pragma unroll
-      for (int o = 16; o; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-      const float x = sigma * dot;
-      const float mn = fmaxf(m[h], x);
-      const float sc = expf(m[h] - mn), p = expf(x - mn);
-      l[h] = fmaf(l[h], sc, p);
+      for (int c = 0; c < 4; ++c) acc[h][c] *= sch;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc[h][c] = fmaf(acc[h][c], sc, p * vv[c]);
-      m[h] = mn;
+      for (int u = 0; u < kBatch; ++u) {
+        const float pu = __shfl_sync(0xffffffffu, p, 4 * u + h);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[h][c] = fmaf(pu, vv[u][c], acc[h][c]);
+      }
     }
   }
 #pragma unroll
