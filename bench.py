@@ -39,8 +39,11 @@ METRIC = "1-bit decode-attention tokens/s and achieved HBM GB/s (n=8192), % of r
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 FALLBACK_HBM_GBS = 6650.0
 CALIB = (True, 0.8, 0.9)
-DECODE_KERNEL_SOURCES = {"octet": "decode_attention_cq_b200/csrc/decode_mma.cu",
-                         "canonical": "decode_attention_cq_b200/csrc/decode_generic.cu"}
+def decode_kernel_source(path: str, bits: int) -> str:
+    """Source file of the kernel that one decode step of this path launches."""
+    if path != "octet":
+        return "decode_attention_cq_b200/csrc/decode_generic.cu"
+    return "decode_attention_cq_b200/csrc/" + ("decode_mma.cu" if bits == 1 else "decode_ring.cu")
 
 
 def algorithmic_bytes(B, Hq, Hkv, n, d, bits, dsize=2):
@@ -68,18 +71,20 @@ def measured_peaks():
 
 
 def traffic_record(path: str, workload: str, bits: int):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    this workload and the kernel source has not changed since."""
+    """DRAM bytes per launch from the committed ncu summaries, if one was taken
+    on this workload and bit width and the kernel source has not changed since."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
+    src = decode_kernel_source(path, bits)
+    digest = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()[:16]
     with open(p) as f:
-        rec = json.load(f).get(path)
-    if not rec or rec.get("workload") != workload or rec.get("bits", 1) != bits:
-        return None
-    src = os.path.join(ROOT, DECODE_KERNEL_SOURCES[path])
-    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return rec if rec.get("source_sha256_16") == digest else None
+        records = json.load(f)["records"]
+    for rec in records:
+        if (rec.get("source") == src and rec.get("workload") == workload and rec.get("bits") == bits
+                and rec.get("source_sha256_16") == digest):
+            return rec
+    return None
 
 
 class ClockSampler:
@@ -311,7 +316,7 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "u1 codes, int8 tensor-core products, f32 softmax, f16 I/O" if args.path == "octet"
+        "dtype": "u%d codes, int8 tensor-core products, f32 softmax, f16 I/O" % bits if args.path == "octet"
         else "u%d codes, f32 math, f16 I/O" % bits,
         "data": "synthetic (seeded InternVL-2.5-shaped K/V caches, no dataset or checkpoint)",
         "config": {"workload": args.workload, "batch_per_gpu": B, "global_batch": B * world,
