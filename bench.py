@@ -39,11 +39,14 @@ METRIC = "1-bit decode-attention tokens/s and achieved HBM GB/s (n=8192), % of r
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 FALLBACK_HBM_GBS = 6650.0
 CALIB = (True, 0.8, 0.9)
-def decode_kernel_source(path: str, bits: int) -> str:
-    """Source file of the kernel that one decode step of this path launches."""
-    if path != "octet":
-        return "decode_attention_cq_b200/csrc/decode_generic.cu"
-    return "decode_attention_cq_b200/csrc/" + ("decode_mma.cu" if bits == 1 else "decode_ring.cu")
+KERNEL_SOURCES = {"k_decode_row": "decode_row.cu", "k_decode_mma": "decode_mma.cu",
+                  "k_decode_octet": "decode_octet.cu", "k_decode_ring": "decode_ring.cu",
+                  "k_scores + k_softmax_v + k_merge": "decode_generic.cu"}
+
+
+def decode_kernel_source(kernel: str) -> str:
+    """Source file of a decode kernel named by cq_decode_kernel_name."""
+    return "decode_attention_cq_b200/csrc/" + KERNEL_SOURCES[kernel]
 
 
 def algorithmic_bytes(B, Hq, Hkv, n, d, bits, dsize=2):
@@ -70,13 +73,13 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def traffic_record(path: str, workload: str, bits: int):
+def traffic_record(kernel: str, workload: str, bits: int):
     """DRAM bytes per launch from the committed ncu summaries, if one was taken
     on this workload and bit width and the kernel source has not changed since."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    src = decode_kernel_source(path, bits)
+    src = decode_kernel_source(kernel)
     digest = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()[:16]
     with open(p) as f:
         records = json.load(f)["records"]
@@ -302,7 +305,8 @@ def run_ours(args, world, rank, local):
     alg = algorithmic_bytes(B, w.hq, w.hkv, n, w.d, bits, dsize) + 2 * B * w.hkv * n_text * w.d * dsize
     kernel_ms = sum(step_ms) / len(step_ms)  # the step's launches (one on the plain octet path)
     achieved = alg / (kernel_ms * 1e-3) / 1e9
-    trec = None if n_text else traffic_record(args.path, args.workload, bits)
+    kernel = cq.cq_decode_kernel_name(*layouts, B, w.hq, w.hkv, n, w.d, bits)
+    trec = None if n_text else traffic_record(kernel, args.workload, bits)
     fill_mean = sum(fill_ms) / len(fill_ms)
     fill_alg = cache_fill_bytes(B, w.hkv, n, w.d, bits)
     line = {
@@ -329,9 +333,7 @@ def run_ours(args, world, rank, local):
                      "frac": achieved / peak, "peak_source": peak_src,
                      "traffic": None if trec is None else trec["dram_bytes_per_launch"],
                      "algorithmic_bytes_per_launch": alg,
-                     "kernel": ("k_scores + k_softmax_v + k_merge" if args.path != "octet"
-                                else ("k_decode_mma" if bits == 1 else f"k_decode_ring<{bits}>")
-                                + (" (partial) + k_text_merge" if n_text else ""))},
+                     "kernel": kernel + (" (partial) + k_text_merge" if n_text else "")},
         "cache_fill": {"ms": fill_mean, "algorithmic_bytes": fill_alg,
                        "achieved_gbs": fill_alg / (fill_mean * 1e-3) / 1e9},
         "e2e": {"value": total_tokens / (e2e_mean * 1e-3), "unit": "tokens/s",

@@ -19,6 +19,7 @@ from .calibq import (  # noqa: F401
     cq_decode_attn_mixed,
     cq_decode_attn_mixed_workspace_size,
     cq_decode_attn_workspace_size,
+    cq_decode_kernel_name,
     cq_dequant,
     cq_quantize_kv,
     cq_quantize_kv_workspace_size,

@@ -30,6 +30,7 @@ ENTRY_POINTS = (
     "cq_quantize_kv",
     "cq_quantize_kv_noalloc",
     "cq_decode_attn_workspace_size",
+    "cq_decode_kernel_name",
     "cq_decode_attn",
     "cq_decode_attn_mixed_workspace_size",
     "cq_decode_attn_mixed",
@@ -56,6 +57,7 @@ _SIGS = {
     "cq_quantize_kv": ([_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P], _I),
     "cq_quantize_kv_noalloc": ([_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P], _I),
     "cq_decode_attn_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
+    "cq_decode_kernel_name": ([_I, _I, _I, _I, _I, _I, _I, _I], ctypes.c_char_p),
     "cq_decode_attn": ([_P, _I, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F,
                         cq_calib, _P, _P, _SZ, _P], _I),
     "cq_decode_attn_mixed_workspace_size": ([_I, _I, _I, ctypes.POINTER(_SZ)], _I),
@@ -188,6 +190,13 @@ def cq_decode_attn_workspace_size(k_layout: int, v_layout: int, B: int, Hq: int,
     _check(load().cq_decode_attn_workspace_size(k_layout, v_layout, B, Hq, Hkv, n, d, bits,
                                                 ctypes.byref(out)), "cq_decode_attn_workspace_size")
     return out.value
+
+
+def cq_decode_kernel_name(k_layout: int, v_layout: int, B: int, Hq: int, Hkv: int, n: int, d: int,
+                          bits: int) -> str | None:
+    """Name of the kernel cq_decode_attn launches for these arguments, or None."""
+    name = load().cq_decode_kernel_name(k_layout, v_layout, B, Hq, Hkv, n, d, bits)
+    return None if name is None else name.decode()
 
 
 def cq_decode_attn(q: torch.Tensor, k: QuantizedCache, v: QuantizedCache, *,

@@ -39,14 +39,54 @@ cq_status check_ptr(const void* p) {
   return CQ_OK;
 }
 
-// CALIBQ_DECODE_KERNEL=tcgen05 routes every octet-layout decode to the tcgen05
-// kernel (otherwise it serves only rows longer than the mma.sync kernel takes).
-bool force_tcgen05() {
-  static const int forced = [] {
+// 1-bit octet-layout decode kernels: "row" (one CTA per row, logits in tensor
+// memory, n <= 8192), "cluster" (a cluster of CTAs per row, n <= 32768) and
+// "tcgen05" (5th-generation tensor cores, n <= 65536). CALIBQ_DECODE_KERNEL
+// names one to use wherever it supports n; otherwise the choice is the row
+// kernel when it supports n and the batch gives every SM a row, else the
+// cluster kernel, else the tcgen05 one.
+enum class Kernel1 { kAuto, kRow, kCluster, kTcgen05 };
+
+Kernel1 forced_kernel() {
+  static const Kernel1 forced = [] {
     const char* v = getenv("CALIBQ_DECODE_KERNEL");
-    return (v != nullptr && strcmp(v, "tcgen05") == 0) ? 1 : 0;
+    if (v == nullptr) return Kernel1::kAuto;
+    if (strcmp(v, "row") == 0) return Kernel1::kRow;
+    if (strcmp(v, "cluster") == 0) return Kernel1::kCluster;
+    if (strcmp(v, "tcgen05") == 0) return Kernel1::kTcgen05;
+    return Kernel1::kAuto;
   }();
-  return forced != 0;
+  return forced;
+}
+
+int sm_count() {
+  static const int count = [] {
+    int dev = 0, c = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) !=
+                                                   cudaSuccess)
+      return 0;
+    return c;
+  }();
+  return count;
+}
+
+Kernel1 choose_1bit(int n, int rows, bool partial) {
+  const Kernel1 f = forced_kernel();
+  if (f == Kernel1::kRow && cq::decode_row_supports(n)) return Kernel1::kRow;
+  if (f == Kernel1::kCluster && cq::decode_mma_supports(n)) return Kernel1::kCluster;
+  if (f == Kernel1::kTcgen05 && !partial) return Kernel1::kTcgen05;
+  if (cq::decode_row_supports(n) && rows >= sm_count()) return Kernel1::kRow;
+  if (cq::decode_mma_supports(n)) return Kernel1::kCluster;
+  return partial ? Kernel1::kAuto : Kernel1::kTcgen05;  // kAuto: none
+}
+
+cudaError_t launch_decode_1bit(const cq::DecodeArgs& a, cq_dtype dt, cudaStream_t s) {
+  switch (choose_1bit(a.n, a.B * a.Hkv, a.part_o != nullptr)) {
+    case Kernel1::kRow: return cq::launch_decode_row(a, dt, s);
+    case Kernel1::kCluster: return cq::launch_decode_mma(a, dt, s);
+    case Kernel1::kTcgen05: return cq::launch_decode_octet(a, dt, s);
+    default: return cudaErrorNotSupported;
+  }
 }
 
 #define CQ_TRY(expr)                 \
@@ -192,6 +232,22 @@ cq_status cq_decode_attn_workspace_size(cq_layout k_layout, cq_layout v_layout, 
   return CQ_ERR_UNSUPPORTED;
 }
 
+const char* cq_decode_kernel_name(cq_layout k_layout, cq_layout v_layout, int B, int Hq, int Hkv, int n, int d,
+                                  int bits) {
+  if (check_shape(B, Hq, n, d, bits) != CQ_OK || Hkv < 1 || Hq % Hkv) return nullptr;
+  const int G = Hq / Hkv;
+  if (k_layout == CQ_LAYOUT_CANONICAL && v_layout == CQ_LAYOUT_CANONICAL)
+    return G <= 32 ? "k_scores + k_softmax_v + k_merge" : nullptr;
+  if (k_layout != CQ_LAYOUT_OCTET_K || v_layout != CQ_LAYOUT_OCTET_V || G != 4) return nullptr;
+  if (bits != 1) return cq::decode_ring_supports(n, bits) ? "k_decode_ring" : nullptr;
+  if (n > 65536) return nullptr;
+  switch (choose_1bit(n, B * Hkv, false)) {
+    case Kernel1::kRow: return "k_decode_row";
+    case Kernel1::kCluster: return "k_decode_mma";
+    default: return "k_decode_octet";
+  }
+}
+
 cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, const void* k_alpha,
                          const void* k_scale, cq_layout k_layout, const uint8_t* v_codes,
                          const void* v_alpha, const void* v_scale, cq_layout v_layout, int B,
@@ -225,9 +281,7 @@ cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, con
     CQ_TRY(check_ptr(workspace));
     return cuda_status(cq::launch_decode_generic(a, dt, workspace, s));
   }
-  const cudaError_t e = bits != 1 ? cq::launch_decode_ring(a, dt, s)
-                        : (cq::decode_mma_supports(n) && !force_tcgen05()) ? cq::launch_decode_mma(a, dt, s)
-                                                                            : cq::launch_decode_octet(a, dt, s);
+  const cudaError_t e = bits != 1 ? cq::launch_decode_ring(a, dt, s) : launch_decode_1bit(a, dt, s);
   if (e == cudaErrorNotSupported) return CQ_ERR_UNSUPPORTED;
   return cuda_status(e);
 }
@@ -267,7 +321,7 @@ cq_status cq_decode_attn_mixed(const void* q, cq_dtype dt, const uint8_t* k_code
   a.part_o = static_cast<float*>(workspace);
   a.part_lse = a.part_o + (size_t)B * Hq * kD;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = bits != 1 ? cq::launch_decode_ring(a, dt, s) : cq::launch_decode_mma(a, dt, s);
+  cudaError_t e = bits != 1 ? cq::launch_decode_ring(a, dt, s) : launch_decode_1bit(a, dt, s);
   if (e == cudaErrorNotSupported) return CQ_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return CQ_ERR_CUDA;
   return cuda_status(cq::launch_text_merge(a, dt, k_text, v_text, n_text, s));

@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(kThreads) k_scores(DecodeArgs a, Ws ws) {
     const int h = e / kD, j = e % kD;
     sW[h][j] = a.sigma * DT<T>::f(q[(size_t)h * kD + j]) * DT<T>::f(sc[j]);
   }
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31, warp = __shfl_sync(0xffffffffu, (int)threadIdx.x >> 5, 0);  // warp-uniform
   for (int h = warp; h < G; h += kThreads / 32) {
     float s = 0.f;
     for (int j = lane; j < kD; j += 32) s += DT<T>::f(q[(size_t)h * kD + j]) * DT<T>::f(al[j]);
@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(kThreads) k_softmax_v(DecodeArgs a, Ws ws) {
   }
   __syncthreads();
   // sum of weights of this chunk
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31, warp = __shfl_sync(0xffffffffu, (int)threadIdx.x >> 5, 0);  // warp-uniform
   for (int h = warp; h < G; h += kThreads / 32) {
     float s = 0.f;
     for (int u = lane; u < kChunk; u += 32) s += sP[h][u];

@@ -93,7 +93,9 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
   uint8_t* sFrag = sK;                         // weight-limb A fragments, tile lt at bytes [4096 lt, ...)
   float* sPart = reinterpret_cast<float*>(sV);  // per warp-pair partial sums (after the V side)
 
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31, g = lane >> 2, tq = lane & 3;
+  // warp index broadcast from lane 0: known warp-uniform, so shuffles under branches and
+  // loops on it need no reconvergence
+  const int t = threadIdx.x, warp = __shfl_sync(0xffffffffu, t >> 5, 0), lane = t & 31, g = lane >> 2, tq = lane & 3;
   const uint32_t rank = tc::cluster_rank();
   const int row = blockIdx.x / cl;
   const int b = row / a.Hkv, hkv = row % a.Hkv;
@@ -141,23 +143,27 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
   const T* sRows = reinterpret_cast<const T*>(F.stage);  // q[4][kD], alpha_K, s_K, alpha_V, s_V
   wait_copies(&F.bar_rows, 0, err);
   float w[kG];
-  if (t < kD) {
-    const float ak = DT<T>::f(sRows[4 * kD + t]);
-    const float sk = DT<T>::f(sRows[5 * kD + t]);
+  // Every warp runs this (warps 4..7 repeat channels 0..127 and store nothing):
+  // a shuffle the compiler cannot prove convergent, e.g. under a branch on the
+  // thread index, costs several times its latency.
+  {
+    const int ch = t & (kD - 1);
+    const float ak = DT<T>::f(sRows[4 * kD + ch]);
+    const float sk = DT<T>::f(sRows[5 * kD + ch]);
 #pragma unroll
     for (int h = 0; h < kG; ++h) {
-      const float qv = DT<T>::f(sRows[h * kD + t]);
+      const float qv = DT<T>::f(sRows[h * kD + ch]);
       w[h] = a.sigma * qv * sk;
       const float amax = warp_max(fabsf(w[h]));
       const float qa = warp_sum(qv * ak);
-      if (lane == 0) {
+      if (lane == 0 && warp < kD / 32) {
         F.red[warp][h][0] = amax;
         F.red[warp][h][1] = qa;
       }
     }
   }
   __syncthreads();
-  if (t < kD) {
+  if (warp < kD / 32) {  // t < kD
 #pragma unroll
     for (int h = 0; h < kG; ++h) {
       const float amax = fmaxf(fmaxf(F.red[0][h][0], F.red[1][h][0]), fmaxf(F.red[2][h][0], F.red[3][h][0]));

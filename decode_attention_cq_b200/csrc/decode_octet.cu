@@ -112,7 +112,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   Smem& S = *reinterpret_cast<Smem*>(smem_raw);
   float* scores = reinterpret_cast<float*>(smem_raw + align1k(sizeof(Smem)));  // [kG][slice_tokens]
 
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  // warp index broadcast from lane 0: known warp-uniform, so shuffles under branches and
+  // loops on it need no reconvergence
+  const int t = threadIdx.x, warp = __shfl_sync(0xffffffffu, t >> 5, 0), lane = t & 31;
   const uint32_t rank = tc::cluster_rank();
   const int row = blockIdx.x / cl;  // b * Hkv + g
   const int b = row / a.Hkv, g = row % a.Hkv;

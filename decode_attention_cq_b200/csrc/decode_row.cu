@@ -1,0 +1,539 @@
+// Fused 1-bit decode attention, one CTA per (batch, kv-head) row, logits held
+// in tensor memory; register-fed tensor-core MMAs (mma.sync m16n8k32, 8-bit
+// operands, s32 accumulators) over the octet code layouts.
+//
+// Method (CalibQuant article): logits x_i = sigma q.alpha_K + (sigma q (.) s_K)
+// . c^K_i on the integer codes (Method 2, post-scaling), calibration map g on
+// the row's score range (Method 3), softmax, o = alpha_V + s_V (.)
+// sum_i p_i c^V_i / sum_i p_i (Method 2 applied to V).
+//
+// Why one CTA per row: the calibration slope needs the range of ALL logits of
+// the row before any softmax weight exists. Splitting a row over a cluster
+// makes every slice wait twice on its peers (range, then partial sums); here
+// the range is a barrier inside the CTA. The row's logits (n x 4 heads x 4 B,
+// 128 KB at n = 8192) do not fit next to a code ring in shared memory for two
+// CTAs per SM, so they live in tensor memory (256 columns per CTA, two CTAs
+// per SM), written and read back by the thread that owns them.
+//
+// Tiles of 256 tokens (32 octets), 8 warps, two CTAs per SM:
+//  1. one thread copies the q / alpha / s rows and the first chunks of codes;
+//     the K codes and after them the V codes stream through a ring of 16 KB
+//     slots (4 tiles each; tensor copies with the 128-byte swizzle, completing
+//     on a full mbarrier per slot, every wait bounded). A shared counter per
+//     slot collects the warps' releases, and the warp whose release empties
+//     the slot issues the copy that reuses it: no thread waits for a slot;
+//  2. the weights w_h = sigma q_h (.) s_K become 22-bit fixed point in three
+//     int8 limbs, held as the A operand: rows 4 l + h (limb l, head h);
+//  3. K side: warp w takes tiles w, w + 8, ...; B = the codes of 8 octets x 32
+//     channels, masked to bit k (one octet byte holds 8 tokens of a channel;
+//     masking bit k leaves "code of token 8 o + k times 2^k"). The octet each
+//     B column stands for is chosen so that the thread holding D rows g, g + 8
+//     and columns 2 tq, 2 tq + 1 of the four N = 8 tiles ends up with head
+//     g % 4 of octets 4 tq + i and 16 + 4 tq + i (i = 0..3): exactly the
+//     tokens whose softmax weights it needs for the V side's A fragment. Bits
+//     are taken in pairs (k, k + 1); after one exchange between lanes l and
+//     l ^ 16 (the lanes holding limbs 0, 2 and limb 1 of one head), lane l < 16
+//     owns bit k and lane l + 16 bit k + 1. Each lane stores its 8 logits per
+//     bit pair in its own tensor-memory lane;
+//  4. the row range per head (warp shuffles + one CTA barrier) gives the
+//     calibration slope;
+//  5. V side: warp pair (q, q + 4) takes tiles q, q + 4, ... and splits the 128
+//     channels. Per tile a lane reads back its 32 logits, forms P = p 2^(31-k)
+//     for its bit of every pair, swaps them with lane ^ 16 and assembles the A
+//     fragment (rows 4 limb + head, columns octets) with byte permutes;
+//     B = V codes of 8 channels masked to bit k. Sum_l 2^(8l-31) D_l = sum c p;
+//  6. the four warp pairs' sums meet in shared memory; o = alpha_V + s_V (.)
+//     sum c p / sum p.
+// One launch per decode step, no workspace; n <= 8192 tokens per row.
+#include <float.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "mma_util.cuh"
+#include "tc.cuh"
+
+namespace cq {
+
+namespace {
+
+using namespace mu;
+
+constexpr int kThreads = 256;  // 8 warps
+constexpr int kTile = 256;              // tokens per tile (32 octets, 4 KB of codes per side)
+constexpr int kChunkTiles = 4;          // tiles per ring slot
+constexpr int kChunkBytes = kChunkTiles * 4096;
+constexpr int kSlots = 4;
+constexpr int kMaxTiles = 32;  // n <= 8192: 8 tiles per tensor-memory lane quarter, 256 columns
+constexpr int kWMax = (1 << 21) - 1;
+constexpr int kLimbRow = 132;  // bytes per limb row (padding spreads the fragment loads over banks)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kMinSmem = 80 * 1024;  // > 228 KB / 3: at most two CTAs (2 x 256 columns) per SM
+
+struct RowFixed {
+  alignas(16) uint8_t stage[8 * kD * 4];  // q of the 4 heads, alpha_K, s_K, alpha_V, s_V (dtype T)
+  uint64_t full[kSlots], bar_rows;
+  uint32_t released[kSlots];  // warp releases of each slot so far (8 per use)
+  uint32_t uses[kSlots];      // copies issued into each slot so far
+  int err;                    // a bounded wait ran out
+  uint32_t tmem_base;  // written by tcgen05.alloc
+  uint8_t limb[kG * 3][kLimbRow];  // weight limbs: row 3 h + l, byte = channel
+  float red[8][kG][2];             // per-warp reduction scratch
+  float lsum[8][kG];               // per warp: sum of its softmax weights
+  float c0[kG], kscale[kG], alog2[kG], ref[kG], cst[kG];
+  // V-side A fragments of one tile, per warp pair, double-buffered by tile:
+  // [pair][buffer][bit][lane][4 words]; afterwards the pairs' partial sums
+  // [pair][head][channel] (fp32) reuse the space
+  alignas(16) uint32_t frag[4][2][8][32][4];
+};
+static_assert(sizeof(float) * 4 * kG * kD <= sizeof(uint32_t) * 4 * 2 * 8 * 32 * 4, "partial sums fit");
+
+__host__ __device__ constexpr size_t row_smem_bytes() {
+  return (size_t)kSlots * kChunkBytes + sizeof(RowFixed) + 1024;  // + alignment to the swizzle atom
+}
+
+
+// Byte l of each of p0..p3 -> one word (column order), and byte l + 2 -> another.
+__device__ __forceinline__ void gather_limbs(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t p3, uint32_t sel,
+                                             uint32_t& lo, uint32_t& hi) {
+  const uint32_t t01 = __byte_perm(p0, p1, sel), t23 = __byte_perm(p2, p3, sel);
+  lo = __byte_perm(t01, t23, 0x5410);
+  hi = __byte_perm(t01, t23, 0x7632);
+}
+
+// Octet (0..31 within a tile) of a lane's value i (0..7): 4 tq + i, then 16 + 4 tq + i - 4.
+__device__ __forceinline__ int lane_octet(int tq, int i) { return (i < 4) ? 4 * tq + i : 12 + 4 * tq + i; }
+
+// Chunk gi (0 .. 2 nchunk - 1) of the ring: the K codes of tiles 4 gi .. 4 gi + 3,
+// then (gi >= nchunk) the V codes of tiles 4 (gi - nchunk) ..; it lands in slot
+// gi % kSlots. Tiles past the row's end arrive as zeros (tensor-copy bounds fill).
+__device__ __forceinline__ void issue_chunk(RowFixed& F, uint8_t* ring, const CUtensorMap* kmap,
+                                            const CUtensorMap* vmap, int row, int nchunk, int gi) {
+  const int s = gi % kSlots;
+  atomicAdd(&F.uses[s], 1u);
+  tc::mbar_arrive_expect_tx(&F.full[s], kChunkBytes);
+  uint8_t* dst = ring + (size_t)s * kChunkBytes;
+  if (gi < nchunk)
+    tc::tma_load_3d(dst, kmap, 0, gi * kChunkTiles * 32, row, &F.full[s]);
+  else
+    tc::tma_load_3d(dst, vmap, 0, (gi - nchunk) * kChunkTiles * 32, row, &F.full[s]);
+}
+
+// A warp is done reading chunk gi (its share of the slot's 8 releases is
+// `share`); the warp that completes the slot's releases issues the chunk that
+// reuses it, so no thread ever waits for a slot to drain.
+__device__ __forceinline__ void release_chunk(RowFixed& F, uint8_t* ring, const CUtensorMap* kmap,
+                                              const CUtensorMap* vmap, int row, int nchunk, int gi,
+                                              uint32_t share) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) {
+    const int s = gi % kSlots;
+    __threadfence_block();  // this warp's reads of the slot come before the release
+    const uint32_t done = atomicAdd(&F.released[s], share) + share;
+    if (done == 8u * (uint32_t)(gi / kSlots + 1) && gi + kSlots < 2 * nchunk) {
+      __threadfence_block();
+      tc::fence_proxy_async();
+      issue_chunk(F, ring, kmap, vmap, row, nchunk, gi + kSlots);
+    }
+  }
+}
+
+// kmap: K codes as [rows][octets][128 B]; vmap: V codes as [rows][tiles * 32][128 B]
+// (a 128-byte line holds 4 channels' 32 bytes of a tile). Both with the
+// 128-byte swizzle: 16-byte chunk c of line l lands at chunk c ^ (l & 7).
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 2)
+    k_decode_row(const __grid_constant__ DecodeArgs a, uint32_t tmem_cols, const __grid_constant__ CUtensorMap kmap,
+                 const __grid_constant__ CUtensorMap vmap) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* ring = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  RowFixed& F = *reinterpret_cast<RowFixed*>(ring + (size_t)kSlots * kChunkBytes);
+  const uint32_t ring_u = tc::smem_u32(ring);
+
+  // the warp index broadcast from lane 0 is known to be warp-uniform, so branches
+  // and loops on it keep the warp converged: shuffles inside them stay cheap
+  const int t = threadIdx.x, warp = __shfl_sync(0xffffffffu, t >> 5, 0), lane = t & 31, g = lane >> 2, tq = lane & 3;
+  const int row = blockIdx.x, b = row / a.Hkv, hkv = row % a.Hkv;
+  const int n = a.n;
+  const int nt = (n + kTile - 1) / kTile;                   // tiles of the row
+  const int nchunk = (nt + kChunkTiles - 1) / kChunkTiles;  // ring chunks per side
+  volatile int* err = &F.err;
+
+  // ---- 1. barriers, tensor memory, the query and statistics rows, the first chunks
+  if (t == 0) {
+    F.err = 0;
+    for (int s = 0; s < kSlots; ++s) {
+      tc::mbar_init(&F.full[s], 1);
+      F.released[s] = 0;
+      F.uses[s] = 0;
+    }
+    tc::mbar_init(&F.bar_rows, 1);
+    tc::fence_mbar_init();
+    constexpr uint32_t kRow = kD * sizeof(T);
+    const uint8_t* qrow = static_cast<const uint8_t*>(a.q) + ((size_t)b * a.Hq + (size_t)kG * hkv) * kRow;
+    const size_t stat = (size_t)row * kRow;
+    tc::mbar_arrive_expect_tx(&F.bar_rows, 8 * kRow);
+    tc::bulk_load(F.stage, qrow, kG * kRow, &F.bar_rows);
+    tc::bulk_load(F.stage + 4 * kRow, static_cast<const uint8_t*>(a.k_alpha) + stat, kRow, &F.bar_rows);
+    tc::bulk_load(F.stage + 5 * kRow, static_cast<const uint8_t*>(a.k_scale) + stat, kRow, &F.bar_rows);
+    tc::bulk_load(F.stage + 6 * kRow, static_cast<const uint8_t*>(a.v_alpha) + stat, kRow, &F.bar_rows);
+    tc::bulk_load(F.stage + 7 * kRow, static_cast<const uint8_t*>(a.v_scale) + stat, kRow, &F.bar_rows);
+    for (int gi = 0; gi < kSlots && gi < 2 * nchunk; ++gi) issue_chunk(F, ring, &kmap, &vmap, row, nchunk, gi);
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(&F.tmem_base, tmem_cols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = F.tmem_base;
+
+  {
+    // ---- 2. post-scaled K weights w_h = sigma q_h (.) s_K in 22-bit fixed point
+    const T* sRows = reinterpret_cast<const T*>(F.stage);  // q[4][kD], alpha_K, s_K, alpha_V, s_V
+    warp_wait_copies(&F.bar_rows, 0, err);
+    float w[kG];
+    // Every warp runs this (warps 4..7 repeat channels 0..127 and store nothing):
+    // a shuffle the compiler cannot prove convergent, e.g. under a branch on the
+    // thread index, costs several times its latency.
+    {
+      const int ch = t & (kD - 1);
+      const float ak = DT<T>::f(sRows[4 * kD + ch]);
+      const float sk = DT<T>::f(sRows[5 * kD + ch]);
+#pragma unroll
+      for (int h = 0; h < kG; ++h) {
+        const float qv = DT<T>::f(sRows[h * kD + ch]);
+        w[h] = a.sigma * qv * sk;
+        const float amax = warp_max(fabsf(w[h]));
+        const float qa = warp_sum(qv * ak);
+        if (lane == 0 && warp < kD / 32) {
+          F.red[warp][h][0] = amax;
+          F.red[warp][h][1] = qa;
+        }
+      }
+    }
+    __syncthreads();
+    if (warp < kD / 32) {  // t < kD
+#pragma unroll
+      for (int h = 0; h < kG; ++h) {
+        const float amax = fmaxf(fmaxf(F.red[0][h][0], F.red[1][h][0]), fmaxf(F.red[2][h][0], F.red[3][h][0]));
+        const float ks = amax * (1.f / (float)kWMax);  // any scale works: w is rounded with this one
+        const float inv = ks > 0.f ? __frcp_rn(ks) : 0.f;
+        const int wi = max(-kWMax, min(kWMax, __float2int_rn(w[h] * inv)));
+        F.limb[3 * h + 0][t] = (uint8_t)(wi & 127);
+        F.limb[3 * h + 1][t] = (uint8_t)((wi >> 7) & 127);
+        F.limb[3 * h + 2][t] = (uint8_t)((wi >> 14) & 255);
+        if (t == h) {
+          F.kscale[h] = ks;
+          F.c0[h] = a.sigma * (F.red[0][h][1] + F.red[1][h][1] + F.red[2][h][1] + F.red[3][h][1]);
+        }
+      }
+    }
+    __syncthreads();
+
+    // A fragments of the K side, per 32-channel chunk c: row g = (limb g / 4,
+    // head g % 4), row g + 8 = (limb 2, head g) for g < 4, zero for g >= 4.
+    const bool lo = lane < 16;  // lo lanes hold limbs 0 and 2 of head g, hi lanes limb 1 of head g - 4
+    const int h = g & 3;        // the head of every value this lane holds
+    uint32_t wa[4][4];
+    {
+      const uint8_t* r0 = F.limb[3 * h + (g >> 2)];
+      const uint8_t* r1 = F.limb[3 * h + 2];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int j = 32 * c + 4 * tq;
+        wa[c][0] = *reinterpret_cast<const uint32_t*>(r0 + j);
+        wa[c][1] = lo ? *reinterpret_cast<const uint32_t*>(r1 + j) : 0u;
+        wa[c][2] = *reinterpret_cast<const uint32_t*>(r0 + j + 16);
+        wa[c][3] = lo ? *reinterpret_cast<const uint32_t*>(r1 + j + 16) : 0u;
+      }
+    }
+    const float c0 = F.c0[h], kscale = F.kscale[h];
+    const uint32_t tlane = tmem + ((uint32_t)(32 * (warp & 3)) << 16);  // this warp's lane quarter
+
+    // ---- 3. K side: chunk c's tile 4 c + (warp & 3) belongs to warp (4 c + (warp & 3)) % 8
+    float mn = FLT_MAX, mx = -FLT_MAX;  // logit range of head h over this lane's tokens
+    // Every warp runs every pass (a shuffle inside a loop whose trip count the
+    // compiler sees as per-thread costs several times its latency); a pass
+    // without a tile computes on zero codes and stores nothing.
+    for (int pass = 0; pass < nchunk; pass += 2) {
+      const int c = pass + (warp >> 2), s = c % kSlots, j = kChunkTiles * c + (warp & 3);
+      const bool act = c < nchunk, have = act && j < nt;
+      if (act) warp_wait_copies(&F.full[s], (uint32_t)(c / kSlots) & 1u, err);
+      uint32_t bk[4][4][2];  // [32-channel chunk][N tile][reg]
+      if (have) {
+        // lane provides row (lane & 7) of matrix lane >> 3; matrix (N tile 2x + m / 2, half m % 2)
+        const uint32_t tile_u = ring_u + (uint32_t)(s * kChunkBytes + (warp & 3) * 4096);
+        const int m = lane >> 3, r = lane & 7;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const int jn = 2 * x + (m >> 1);
+          const int oct = 2 * jn + 12 * (jn >> 1) + 4 * (r >> 1) + (r & 1);  // octet of B column r
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t rr[4];
+            ldsm_x4(tile_u + oct * 128 + (((2 * cc + (m & 1)) ^ (oct & 7)) << 4), rr);
+            bk[cc][2 * x][0] = rr[0];
+            bk[cc][2 * x][1] = rr[1];
+            bk[cc][2 * x + 1][0] = rr[2];
+            bk[cc][2 * x + 1][1] = rr[3];
+          }
+        }
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+          for (int jn = 0; jn < 4; ++jn) bk[cc][jn][0] = bk[cc][jn][1] = 0u;
+      }
+      if (act) release_chunk(F, ring, &kmap, &vmap, row, nchunk, c, 2);  // K side: four warps per chunk
+      const bool ragged = kTile * (j + 1) > n;
+      const uint32_t col0 = tlane + (uint32_t)(32 * (j >> 2));
+#pragma unroll
+      for (int kp = 0; kp < 4; ++kp) {
+        int d[2][4][4];  // [bit 2 kp + kk][N tile][reg]
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+          for (int jn = 0; jn < 4; ++jn) d[kk][jn][0] = d[kk][jn][1] = d[kk][jn][2] = d[kk][jn][3] = 0;
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint32_t msk = 0x01010101u << (2 * kp + kk);
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+            for (int jn = 0; jn < 4; ++jn) mma_s8u8(d[kk][jn], wa[cc], bk[cc][jn][0] & msk, bk[cc][jn][1] & msk);
+        }
+        // lo lanes finish bit 2 kp, hi lanes bit 2 kp + 1: x = D0 + 2^7 D1 + 2^14 D2
+        const int kown = 2 * kp + (lo ? 0 : 1);
+        const float sc = kscale * __int_as_float((127 - kown) << 23);  // step * 2^-k
+        uint32_t out[8];
+#pragma unroll
+        for (int jn = 0; jn < 4; ++jn)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int i = 2 * jn + e;
+            const int send =
+                lo ? __float_as_int(fmaf(16384.f, (float)d[1][jn][2 + e], (float)d[1][jn][e])) : d[0][jn][e];
+            const int recv = __shfl_xor_sync(0xffffffffu, send, 16);
+            float x;
+            if (lo) {
+              const int d01 = d[0][jn][e] + (recv << 7);  // |d01| < 2^29
+              x = fmaf(16384.f, (float)d[0][jn][2 + e], (float)d01);
+            } else {
+              x = fmaf(128.f, (float)d[1][jn][e], __int_as_float(recv));
+            }
+            const float xl = fmaf(x, sc, c0);
+            if (!ragged || kTile * j + 8 * lane_octet(tq, i) + kown < n) {
+              mn = fminf(mn, xl);
+              mx = fmaxf(mx, xl);
+            }
+            out[i] = __float_as_uint(xl);
+          }
+        if (have) tc::st_x8(col0 + 8 * kp, out);
+      }
+    }
+    tc::wait_st();
+
+    // ---- 4. logit range of the row, calibration slope
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 16));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    if (lo && tq == 0) {
+      F.red[warp][g][0] = mn;
+      F.red[warp][g][1] = mx;
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (t < kG) {
+      float m = FLT_MAX, M = -FLT_MAX;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        m = fminf(m, F.red[q][t][0]);
+        M = fmaxf(M, F.red[q][t][1]);
+      }
+      float slope = 1.f, cst = 0.f;
+      if (a.calib && M > m) {
+        slope = (a.tau_hi * M - a.tau_lo * m) / (M - m);
+        cst = a.tau_lo * m - slope * m;  // g(x) = slope x + cst
+      }
+      F.alog2[t] = slope * kLog2e;
+      F.ref[t] = fmaxf(slope * m, slope * M) * kLog2e;
+      F.cst[t] = cst;
+    }
+    __syncthreads();
+
+    // ---- 5. V side: pair q = warp & 3 takes tiles q, q + 4, ...; hc = warp >> 2 picks
+    // channels 64 hc .. 64 hc + 63 and forms the weight fragments of bits 4 hc .. 4 hc + 3
+    const int q = warp & 3, hc = warp >> 2;
+    const float alog2 = F.alog2[h], ref = F.ref[h];
+    const uint32_t sel = lo ? 0x6240u : 0x7351u;  // bytes (limb, limb + 2) of two words: limbs 0, 2 or 1, 3
+    const uint32_t frag_u = tc::smem_u32(&F.frag[q][0][0][0][0]) + (uint32_t)lane * 16;
+    int acc[8][4];
+#pragma unroll
+    for (int jn = 0; jn < 8; ++jn) acc[jn][0] = acc[jn][1] = acc[jn][2] = acc[jn][3] = 0;
+    float lsum = 0.f;
+    int buf = 0;
+    for (int c = 0; c < nchunk; ++c) {
+      const int gi = nchunk + c, s = gi % kSlots, j = kChunkTiles * c + q;
+      warp_wait_copies(&F.full[s], (uint32_t)(gi / kSlots) & 1u, err);
+      uint32_t bv[8][2];
+      const bool have = j < nt;
+      if (have) {
+        const uint32_t tile_u = ring_u + (uint32_t)(s * kChunkBytes + q * 4096);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const int mat = lane >> 3, half = mat & 1;
+          const int ch = 64 * hc + 16 * p + 8 * (mat >> 1) + (lane & 7);
+          uint32_t r[4];
+          ldsm_x4(tile_u + (ch >> 2) * 128 + (((((ch & 3) << 1) | half) ^ ((ch >> 2) & 7)) << 4), r);
+          bv[2 * p][0] = r[0];
+          bv[2 * p][1] = r[1];
+          bv[2 * p + 1][0] = r[2];
+          bv[2 * p + 1][1] = r[3];
+        }
+      } else {
+#pragma unroll
+        for (int jn = 0; jn < 8; ++jn) bv[jn][0] = bv[jn][1] = 0u;
+      }
+      release_chunk(F, ring, &kmap, &vmap, row, nchunk, gi, 1);  // V side: all eight warps per chunk
+      // no skip for a missing tile (zero codes, zero weights): the shuffles below
+      // stay out of branches on the warp index
+      const bool ragged = kTile * (j + 1) > n;  // true for a missing tile: every token masked
+      uint32_t xs[16];  // logits of bit pairs 2 hc, 2 hc + 1 (this lane's bit of each)
+      tc::ld_x16(tlane + (uint32_t)(32 * (j >> 2) + 16 * hc), xs);
+      tc::wait_ld();
+      const uint32_t fbuf = frag_u + (uint32_t)buf * 4096;
+#pragma unroll
+      for (int kq = 0; kq < 2; ++kq) {
+        const int kp = 2 * hc + kq, kown = 2 * kp + (lo ? 0 : 1);
+        const float bias = (float)(31 - kown) - ref;
+        const float unscale = __int_as_float((127 - 31 + kown) << 23);  // 2^(k - 31)
+        uint32_t pown[8], poth[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float p = ex2_approx(fmaf(__uint_as_float(xs[8 * kq + i]), alog2, bias));
+          const bool ok = !ragged || kTile * j + 8 * lane_octet(tq, i) + kown < n;
+          pown[i] = ok ? __float2uint_rn(p) : 0u;
+          lsum = ok ? fmaf(p, unscale, lsum) : lsum;
+          poth[i] = __shfl_xor_sync(0xffffffffu, pown[i], 16);
+        }
+        // bit 2 kp: the lo lanes' weights; bit 2 kp + 1: the hi lanes'
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          uint32_t P[8], af[4];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) P[i] = ((kk == 0) == lo) ? pown[i] : poth[i];
+          gather_limbs(P[0], P[1], P[2], P[3], sel, af[0], af[1]);
+          gather_limbs(P[4], P[5], P[6], P[7], sel, af[2], af[3]);
+          sts128(fbuf + (uint32_t)(2 * kp + kk) * 512, af);
+        }
+      }
+      tc::bar_sync(2 + q, 64);  // the pair's weight fragments of this tile are complete
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        uint32_t af[4];
+        lds128(fbuf + (uint32_t)k * 512, af);
+        const uint32_t msk = 0x01010101u << k;
+#pragma unroll
+        for (int jn = 0; jn < 8; ++jn) mma_u8u8(acc[jn], af, bv[jn][0] & msk, bv[jn][1] & msk);
+      }
+      buf ^= 1;
+    }
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+    if (lo && tq == 0) F.lsum[warp][g] = lsum;
+
+    // ---- 6. limbs combined (lane and lane ^ 16), the pairs summed, o written
+    __syncthreads();  // every warp is done with the fragment buffers: the partial sums reuse them
+    float* part = reinterpret_cast<float*>(&F.frag[0][0][0][0][0]);  // [pair][head][channel]
+    {
+      const float s_lo = lo ? 0x1p-31f : 0x1p-23f, s_hi = lo ? 0x1p-15f : 0x1p-7f;
+#pragma unroll
+      for (int jn = 0; jn < 8; ++jn) {
+        float v[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          v[e] = fmaf((float)acc[jn][e + 2], s_hi, (float)acc[jn][e] * s_lo);
+          v[e] += __shfl_xor_sync(0xffffffffu, v[e], 16);
+        }
+        if (lo)
+          *reinterpret_cast<float2*>(part + (q * kG + g) * kD + 64 * hc + 8 * jn + 2 * tq) = make_float2(v[0], v[1]);
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int idx = 2 * t + e, hh = idx >> 7, ch = idx & 127;
+      float sum = 0.f, l = 0.f;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) sum += part[(p * kG + hh) * kD + ch];
+#pragma unroll
+      for (int w8 = 0; w8 < 8; ++w8) l += F.lsum[w8][hh];
+      const float alpha = DT<T>::f(sRows[6 * kD + ch]);
+      const float step = *err ? __int_as_float(0x7fc00000) : DT<T>::f(sRows[7 * kD + ch]);
+      const size_t bh = (size_t)b * a.Hq + (size_t)kG * hkv + hh;
+      if (a.part_o == nullptr) {
+        static_cast<T*>(a.out)[bh * kD + ch] = DT<T>::from_float(fmaf(step, sum / l, alpha));
+      } else {
+        a.part_o[bh * kD + ch] = fmaf(step, sum / l, alpha);
+        // sum_i exp(y_i) = 2^ref sum_i p_i e^cst with p_i = 2^(x_i alog2 - ref)
+        if (ch == 0) a.part_lse[bh] = fmaf(F.ref[hh], 0.6931471805599453f, logf(l)) + F.cst[hh];
+      }
+    }
+  }
+
+  // ---- teardown: tensor memory back; on the error path, copies still in flight land first
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, tmem_cols);
+  }
+  if (t == 0 && *err) {
+    for (int s = 0; s < kSlots; ++s)
+      if (F.uses[s] > 0) tc::mbar_wait(&F.full[s], (F.uses[s] - 1) & 1u, kSpin);
+  }
+}
+
+template <typename T>
+cudaError_t run_row(const DecodeArgs& a, cudaStream_t stream) {
+  const int rows = a.B * a.Hkv;
+  const int nt = (a.n + kTile - 1) / kTile;
+  uint32_t cols = 32;  // tensor-memory columns: 32 per tile of a lane quarter, a power of two >= 32
+  while (cols < 32u * (uint32_t)((nt + 3) / 4)) cols <<= 1;
+  const size_t smem = row_smem_bytes() > (size_t)kMinSmem ? row_smem_bytes() : (size_t)kMinSmem;
+  static bool attr_set = false;  // benign race: every caller sets the same value
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_decode_row<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)  // two CTAs per SM need the largest shared-memory carve-out
+      e = cudaFuncSetAttribute(k_decode_row<T>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  CUtensorMap kmap, vmap;
+  if (!encode_3d(&kmap, a.k_codes, kD, (uint64_t)(a.n + 7) / 8, (uint64_t)rows, kChunkTiles * 32,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_3d(&vmap, a.v_codes, 128, (uint64_t)nt * 32, (uint64_t)rows, kChunkTiles * 32,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  k_decode_row<T><<<rows, kThreads, smem, stream>>>(a, cols, kmap, vmap);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool decode_row_supports(int n) { return n >= 1 && n <= kMaxTiles * kTile; }
+
+cudaError_t launch_decode_row(const DecodeArgs& a, cq_dtype dt, cudaStream_t stream) {
+  if (!decode_row_supports(a.n)) return cudaErrorNotSupported;
+  if (dt == CQ_F16) return run_row<half>(a, stream);
+  return run_row<float>(a, stream);
+}
+
+}  // namespace cq

@@ -53,7 +53,9 @@ __global__ void __launch_bounds__(kThreads) k_text_merge(const T* __restrict__ q
   __shared__ float s_m[kWarps][kG], s_l[kWarps][kG];
   __shared__ float s_acc[kWarps][kG][kD];
   const int row = blockIdx.x, b = row / Hkv, hkv = row % Hkv;
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  // warp index broadcast from lane 0: known warp-uniform, so shuffles under branches and
+  // loops on it need no reconvergence
+  const int t = threadIdx.x, warp = __shfl_sync(0xffffffffu, t >> 5, 0), lane = t & 31;
   const int my_h = lane & 3;  // head of the logit this lane owns after the butterfly
   const size_t bh0 = (size_t)b * Hq + (size_t)kG * hkv;  // first query head of the row
 
@@ -69,7 +71,11 @@ __global__ void __launch_bounds__(kThreads) k_text_merge(const T* __restrict__ q
   }
   const T* kr = kt + (size_t)row * n_text * kD + 4 * lane;
   const T* vr = vt + (size_t)row * n_text * kD + 4 * lane;
-  for (int j0 = kBatch * warp; j0 < n_text; j0 += kBatch * kWarps) {
+  // every warp runs every pass (a pass past the end masks all its tokens): the
+  // butterfly's shuffles must not sit in a loop whose trip count the compiler
+  // sees as per-thread, where each costs several times its latency
+  for (int jb = 0; jb < n_text; jb += kBatch * kWarps) {
+    const int j0 = jb + kBatch * warp;
     float dv[kBatch * kG];  // partial dots, index 4 token + head
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {

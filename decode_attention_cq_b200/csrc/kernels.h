@@ -66,5 +66,9 @@ cudaError_t launch_decode_ring(const DecodeArgs& a, cq_dtype dt, cudaStream_t st
 // ---- decode_mma.cu (octet layouts, bits = 1, Hq = 4 Hkv, n <= 32768, mma.sync)
 bool decode_mma_supports(int n);
 cudaError_t launch_decode_mma(const DecodeArgs& a, cq_dtype dt, cudaStream_t stream);
+// One CTA per (batch, kv-head) row with the logits in tensor memory (1 bit,
+// octet layouts, Hq = 4 Hkv, n <= 8192).
+bool decode_row_supports(int n);
+cudaError_t launch_decode_row(const DecodeArgs& a, cq_dtype dt, cudaStream_t stream);
 
 }  // namespace cq

@@ -28,10 +28,22 @@ __device__ __forceinline__ void lds128(uint32_t addr, uint32_t (&r)[4]) {
                : "memory");
 }
 
+__device__ __forceinline__ void sts128(uint32_t addr, const uint32_t (&r)[4]) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+
 // D += A (16x32 u8, row) x B (32x8 s8, col). Register-only: the compiler may
 // interleave independent MMAs.
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// D += A (16x32 s8, row) x B (32x8 u8, col)
+__device__ __forceinline__ void mma_s8u8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -72,6 +84,15 @@ __device__ __forceinline__ int logit_pos(int unit, int k, int h, int o) {
 // (its outputs become NaN) instead of hanging.
 __device__ __forceinline__ void wait_copies(uint64_t* bar, uint32_t parity, volatile int* err) {
   if (!tc::mbar_wait(bar, parity, kSpin)) *err = 1;
+}
+
+// The same for a whole warp: every lane probes without suspending and the warp
+// leaves together once every lane has seen the phase complete, so no lane
+// trails the others into the next warp-collective instruction.
+__device__ __forceinline__ void warp_wait_copies(uint64_t* bar, uint32_t parity, volatile int* err) {
+  for (uint32_t i = 0; i < kSpin; ++i)
+    if (__all_sync(0xffffffffu, tc::mbar_test_wait(bar, parity))) return;
+  *err = 1;
 }
 
 // ---------------------------------------------------------------- host side

@@ -193,11 +193,10 @@ cq_status cq_decode_attn_workspace_size(cq_layout k_layout, cq_layout v_layout, 
  *   k_alpha, k_scale, v_alpha, v_scale: [B][Hkv][d] in `dt`.
  *
  * Supported layout pairs: (CANONICAL, CANONICAL) for any bits and any Hq/Hkv;
- * (OCTET_K, OCTET_V) for bits = 1, d = 128, Hq = 4*Hkv and n <= 65536 -- the
- * tensor-core path (register-fed MMAs up to n = 32768, tcgen05 beyond; setting
- * the environment variable CALIBQ_DECODE_KERNEL=tcgen05 before the first call
- * selects tcgen05 for every n). Results of the two kernels agree within the
- * output tolerance, not bit for bit.
+ * (OCTET_K, OCTET_V) for d = 128, Hq = 4*Hkv and n <= 65536 at bits = 1
+ * (n <= 32768 at bits 2, 4, 8) -- the tensor-core path, one launch per call.
+ * cq_decode_kernel_name says which kernel a call launches; the 1-bit kernels
+ * agree with each other within the output tolerance, not bit for bit.
  */
 cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, const void* k_alpha,
                          const void* k_scale, cq_layout k_layout, const uint8_t* v_codes,
@@ -205,6 +204,23 @@ cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, con
                          int Hq, int Hkv, int n, int d, int bits, float softmax_scale,
                          cq_calib calib, void* out, void* workspace, size_t ws_bytes,
                          cq_stream_t stream);
+
+/*
+ * Name of the kernel that cq_decode_attn launches for these layouts and sizes
+ * on the current device, or NULL when the call would not launch one (invalid
+ * or unsupported arguments). Host-only; reads the device's SM count once.
+ *   1 bit, octet layouts: "k_decode_row" (one CTA per (sequence, kv-head) row,
+ *     n <= 8192, chosen when B * Hkv >= the SM count), "k_decode_mma" (a
+ *     cluster of CTAs per row, n <= 32768) or "k_decode_octet" (tcgen05,
+ *     n <= 65536). The environment variable CALIBQ_DECODE_KERNEL = row |
+ *     cluster | tcgen05, read once per process, forces one of them wherever it
+ *     supports n.
+ *   2, 4, 8 bits, octet layouts: "k_decode_ring".
+ *   Canonical layouts: "k_scores + k_softmax_v + k_merge" (three launches).
+ * The returned string is static; the caller does not free it.
+ */
+const char* cq_decode_kernel_name(cq_layout k_layout, cq_layout v_layout, int B, int Hq, int Hkv, int n, int d,
+                                  int bits);
 
 /*
  * Workspace of cq_decode_attn_mixed: the visual part's partial result

@@ -78,6 +78,23 @@ def test_size_queries_validate(lib):
     assert cq.cq_quantize_kv_workspace_size(64, 8, 8192, 128) > 0
 
 
+def test_decode_kernel_name_follows_the_documented_choice(lib):
+    K, V, C = cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V, cq.LAYOUT_CANONICAL
+    assert cq.cq_decode_kernel_name(C, C, 2, 8, 2, 1000, 128, 3) is None  # bits
+    assert cq.cq_decode_kernel_name(K, V, 2, 8, 2, 1000, 64, 1) is None  # d
+    assert cq.cq_decode_kernel_name(K, V, 2, 12, 2, 1000, 128, 1) is None  # G = 6
+    assert cq.cq_decode_kernel_name(K, C, 2, 8, 2, 1000, 128, 1) is None  # mixed layouts
+    assert cq.cq_decode_kernel_name(C, C, 2, 12, 2, 1000, 128, 4) == "k_scores + k_softmax_v + k_merge"
+    for bits in (2, 4, 8):
+        assert cq.cq_decode_kernel_name(K, V, 2, 8, 2, 32768, 128, bits) == "k_decode_ring"
+        assert cq.cq_decode_kernel_name(K, V, 2, 8, 2, 32769, 128, bits) is None
+    assert cq.cq_decode_kernel_name(K, V, 64, 32, 8, 8192, 128, 1) in ("k_decode_row", "k_decode_mma")
+    assert cq.cq_decode_kernel_name(K, V, 64, 32, 8, 8193, 128, 1) == "k_decode_mma"
+    assert cq.cq_decode_kernel_name(K, V, 1, 8, 2, 32768, 128, 1) == "k_decode_mma"
+    assert cq.cq_decode_kernel_name(K, V, 1, 8, 2, 32769, 128, 1) == "k_decode_octet"
+    assert cq.cq_decode_kernel_name(K, V, 1, 8, 2, 65537, 128, 1) is None
+
+
 def test_null_pointers_rejected_before_any_cuda_call(lib):
     st = lib.cq_quantize_kv(None, 0, 1, 1, 16, 128, 1, 0, None, None, None, None, 0, None)
     assert st == cq.CQ_ERR_INVALID_ARG

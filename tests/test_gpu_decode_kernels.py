@@ -1,7 +1,9 @@
-"""Both octet-layout decode kernels against the fp64 oracle: the mma.sync
-kernel (default up to n = 32768) and the tcgen05 kernel (rows longer than
-that, or every row when CALIBQ_DECODE_KERNEL=tcgen05), each in a child process
-so that the selection, read once per process, applies."""
+"""The 1-bit octet-layout decode kernels against the fp64 oracle: the
+one-CTA-per-row kernel (n <= 8192, chosen when the batch gives every SM a
+row), the cluster kernel (n <= 32768) and the tcgen05 kernel (longer rows),
+each also forced with CALIBQ_DECODE_KERNEL in a child process so that the
+selection, read once per process, applies. A forced kernel that does not take
+n falls back to the default choice."""
 
 import json
 import os
@@ -15,9 +17,12 @@ from _util import OUT_RTOL
 pytestmark = pytest.mark.gpu
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-CASES = [[1, 1, [True, 0.8, 0.9]], [300, 2, [False, 1.0, 1.0]], [1025, 2, [True, 0.8, 0.9]],
-         [2049, 1, [True, 1.0, 0.5]], [8192, 1, [True, 0.8, 0.9]], [10000, 1, [True, 0.5, 1.0]],
-         [12000, 1, [True, 0.8, 0.9]], [14000, 1, [True, 0.8, 0.9]], [20000, 1, [True, 0.8, 0.9]]]
+CASES = [[1, 1, [True, 0.8, 0.9]], [7, 1, [True, 0.8, 0.9]], [255, 1, [True, 0.8, 0.9]],
+         [256, 1, [False, 1.0, 1.0]], [300, 2, [False, 1.0, 1.0]], [1024, 1, [True, 0.8, 0.9]],
+         [1025, 2, [True, 0.8, 0.9]], [2049, 1, [True, 1.0, 0.5]], [3328, 1, [True, 0.8, 0.9]],
+         [4097, 1, [True, 0.8, 0.9]], [8191, 1, [True, 0.5, 1.0]], [8192, 1, [True, 0.8, 0.9]],
+         [600, 80, [True, 0.8, 0.9]], [10000, 1, [True, 0.5, 1.0]], [12000, 1, [True, 0.8, 0.9]],
+         [14000, 1, [True, 0.8, 0.9]], [20000, 1, [True, 0.8, 0.9]]]
 
 
 def _run(kernel):
@@ -31,7 +36,7 @@ def _run(kernel):
     return json.loads(res.stdout.strip().splitlines()[-1])["errs"]
 
 
-@pytest.mark.parametrize("kernel", [None, "tcgen05"])
+@pytest.mark.parametrize("kernel", [None, "row", "cluster", "tcgen05"])
 def test_octet_kernels_match_oracle(cuda_device, kernel):
     errs = _run(kernel)
     for (n, batch, calib), e in zip(CASES, errs):
