@@ -412,6 +412,105 @@ def run_reference(args, world, rank):
 args_global = None
 
 
+BUDGET_LAYERS, BUDGET_N = 32, 3328  # full InternVL-2.5-8B decode step at n = 3328
+
+
+def budget_batches(budget_gb: float, hkv: int = 8, d: int = 128):
+    """Largest batch whose KV cache fits the budget (GB = 1e9 bytes, cache only):
+    1-bit codes plus f16 alpha / step of K and V, versus an f16 cache."""
+    per_seq_1bit = BUDGET_LAYERS * hkv * (2 * BUDGET_N * d // 8 + 4 * d * 2)
+    per_seq_f16 = BUDGET_LAYERS * hkv * 2 * BUDGET_N * d * 2
+    return int(budget_gb * 1e9 // per_seq_1bit), int(budget_gb * 1e9 // per_seq_f16), per_seq_1bit, per_seq_f16
+
+
+def _time_graph(step, steps: int, warmup: int) -> float:
+    """Mean ms of one captured step (all layers), CUDA events on the capture stream."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            step()
+        for _ in range(warmup):
+            g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(s)
+        for _ in range(steps):
+            g.replay()
+        e1.record(s)
+        e1.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del g
+    return ms
+
+
+def run_budget(args):
+    """Memory-budget sweep: a full 32-layer decode step (32 / 8 heads, d = 128,
+    n = 3328) with the largest batch whose KV cache fits each budget, 1-bit
+    cache through libcalibq against an f16 cache through PyTorch's fused
+    attention (scaled_dot_product_attention, the comparison arm). Every layer
+    has its own buffers (the working set is far above L2). Inputs are random:
+    the step time does not depend on the values. One JSON line per budget."""
+    dev = torch.device("cuda", 0)
+    hq, hkv, d, n = 32, 8, 128, BUDGET_N
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4)
+    for budget in args.budgets:
+        b1, b16, per1, per16 = budget_batches(budget, hkv, d)
+        rb = cq.cq_codes_bytes(cq.LAYOUT_OCTET_K, 1, 1, n, d, 1)  # == the OCTET_V row at n = 3328
+        layers = []
+        for _ in range(BUDGET_LAYERS):
+            codes = [torch.randint(0, 256, (b1, hkv, rb), dtype=torch.uint8, device=dev, generator=gen)
+                     for _ in range(2)]
+            stats = [torch.rand(b1, hkv, d, device=dev, generator=gen).half() + 0.5 for _ in range(4)]
+            kq = cq.QuantizedCache(codes[0], stats[0] - 1.0, stats[1], cq.LAYOUT_OCTET_K, 1, n)
+            vq = cq.QuantizedCache(codes[1], stats[2] - 1.0, stats[3], cq.LAYOUT_OCTET_V, 1, n)
+            q = torch.randn(b1, hq, d, device=dev, generator=gen).half()
+            layers.append((q, kq, vq, torch.empty_like(q)))
+        kernel = cq.cq_decode_kernel_name(cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V, b1, hq, hkv, n, d, 1)
+
+        def step1():
+            for q, kq, vq, out in layers:
+                cq.cq_decode_attn(q, kq, vq, calib=CALIB, out=out)
+
+        steps = min(args.steps, 20)  # a 32-layer step is milliseconds long
+        ms1 = _time_graph(step1, steps, args.warmup)
+        bytes1 = BUDGET_LAYERS * algorithmic_bytes(b1, hq, hkv, n, d, 1)
+        del layers, step1
+        torch.cuda.empty_cache()
+        layers16 = []
+        for _ in range(BUDGET_LAYERS):
+            k = torch.randn(b16, hkv, n, d, device=dev, generator=gen).half()
+            v = torch.randn(b16, hkv, n, d, device=dev, generator=gen).half()
+            q = torch.randn(b16, hq, 1, d, device=dev, generator=gen).half()
+            layers16.append((q, k, v))
+
+        def step16():
+            for q, k, v in layers16:
+                torch.nn.functional.scaled_dot_product_attention(q, k, v, enable_gqa=True)
+
+        ms16 = _time_graph(step16, steps, args.warmup)
+        bytes16 = BUDGET_LAYERS * (2 * b16 * hkv * n * d * 2 + 2 * b16 * hq * d * 2)
+        del layers16, step16
+        torch.cuda.empty_cache()
+        tps1, tps16 = b1 / (ms1 * 1e-3), b16 / (ms16 * 1e-3)
+        print(json.dumps({
+            "metric": "decode-step tokens/s under a KV-cache memory budget (32 layers, n=3328)",
+            "budget_gb": budget, "data": "synthetic (random codes, statistics and f16 caches)",
+            "config": {"workload": "budget_n3328_32layers", "layers": BUDGET_LAYERS, "q_heads": hq, "kv_heads": hkv,
+                       "head_dim": d, "n_tokens": n, "cache_bytes_per_sequence": {"1bit": per1, "f16": per16}},
+            "calibquant_1bit": {"batch": b1, "ms_per_step": ms1, "tokens_per_s": tps1, "kernel": kernel,
+                                "achieved_gbs": bytes1 / (ms1 * 1e-3) / 1e9},
+            "f16_cache": {"batch": b16, "ms_per_step": ms16, "tokens_per_s": tps16,
+                          "kernel": "torch scaled_dot_product_attention (enable_gqa)",
+                          "achieved_gbs": bytes16 / (ms16 * 1e-3) / 1e9},
+            "speedup": tps1 / tps16}), flush=True)
+
+
 def main():
     global args_global
     ap = argparse.ArgumentParser()
@@ -426,10 +525,16 @@ def main():
     ap.add_argument("--text", type=int, default=0,
                     help="full-precision text tokens after the quantized ones (mixed cache)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--budget-sweep", action="store_true",
+                    help="32-layer decode step under KV-cache budgets, 1-bit vs f16 cache (one line per budget)")
+    ap.add_argument("--budgets", type=float, nargs="+", default=[5, 10, 20, 30])
     args = ap.parse_args()
     args_global = args
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.budget_sweep:
+        run_budget(args)
+        return
     world, rank, local = dist_setup()
     if args.impl == "reference":
         line = run_reference(args, world, rank)
