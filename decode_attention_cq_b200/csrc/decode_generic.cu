@@ -72,12 +72,16 @@ __global__ void __launch_bounds__(kThreads) k_scores(DecodeArgs a, Ws ws) {
     sW[h][j] = a.sigma * DT<T>::f(q[(size_t)h * kD + j]) * DT<T>::f(sc[j]);
   }
   const int lane = threadIdx.x & 31, warp = __shfl_sync(0xffffffffu, (int)threadIdx.x >> 5, 0);  // warp-uniform
-  for (int h = warp; h < G; h += kThreads / 32) {
+  // passes over the heads with a trip count from G only: shuffles under a loop
+  // on the warp index cost several times their latency
+  for (int h0 = 0; h0 < G; h0 += kThreads / 32) {
+    const int h = h0 + warp;
     float s = 0.f;
-    for (int j = lane; j < kD; j += 32) s += DT<T>::f(q[(size_t)h * kD + j]) * DT<T>::f(al[j]);
+    if (h < G)
+      for (int j = lane; j < kD; j += 32) s += DT<T>::f(q[(size_t)h * kD + j]) * DT<T>::f(al[j]);
 #pragma unroll
     for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) sc0[h] = a.sigma * s;
+    if (lane == 0 && h < G) sc0[h] = a.sigma * s;
   }
   __syncthreads();
 
@@ -171,12 +175,14 @@ __global__ void __launch_bounds__(kThreads) k_softmax_v(DecodeArgs a, Ws ws) {
   __syncthreads();
   // sum of weights of this chunk
   const int lane = threadIdx.x & 31, warp = __shfl_sync(0xffffffffu, (int)threadIdx.x >> 5, 0);  // warp-uniform
-  for (int h = warp; h < G; h += kThreads / 32) {
+  for (int h0 = 0; h0 < G; h0 += kThreads / 32) {  // trip count from G only (see above)
+    const int h = h0 + warp;
     float s = 0.f;
-    for (int u = lane; u < kChunk; u += 32) s += sP[h][u];
+    if (h < G)
+      for (int u = lane; u < kChunk; u += 32) s += sP[h][u];
 #pragma unroll
     for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) ws.l[(row0 + h) * C + blockIdx.y] = s;
+    if (lane == 0 && h < G) ws.l[(row0 + h) * C + blockIdx.y] = s;
   }
   // sum_i p_i c_ij: thread = (channel j, half of the chunk)
   const int j = threadIdx.x & (kD - 1), half = threadIdx.x >> 7;

@@ -10,6 +10,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace cq {
 
@@ -19,12 +20,10 @@ constexpr int kThreads = 256;
 constexpr int kTpr = kD / 8;            // threads per token row (8 channels each)
 constexpr int kRpi = kThreads / kTpr;   // token rows per iteration
 
+// Per-channel min / max of tokens [i0, i1) of one row; thread j < kD gets
+// channel j's pair. 16 threads cover a token row (8 channels each).
 template <typename T>
-__global__ void __launch_bounds__(kThreads) k_stats(const T* __restrict__ x, int n, int S,
-                                                    float* __restrict__ part) {
-  const int row = blockIdx.x, s = blockIdx.y;
-  const int per = (n + S - 1) / S;
-  const int i0 = s * per, i1 = min(n, i0 + per);
+__device__ __forceinline__ void tile_minmax(const T* __restrict__ xrow, int i0, int i1, float& a, float& b) {
   const int cg = threadIdx.x % kTpr, r = threadIdx.x / kTpr;
   float mn[8], mx[8];
 #pragma unroll
@@ -32,7 +31,8 @@ __global__ void __launch_bounds__(kThreads) k_stats(const T* __restrict__ x, int
     mn[e] = FLT_MAX;
     mx[e] = -FLT_MAX;
   }
-  const T* base = x + (size_t)row * n * kD + cg * 8;
+  const T* base = xrow + cg * 8;
+#pragma unroll 4
   for (int i = i0 + r; i < i1; i += kRpi) {
     float v[8];
     load8(base + (size_t)i * kD, v);
@@ -49,28 +49,40 @@ __global__ void __launch_bounds__(kThreads) k_stats(const T* __restrict__ x, int
     smx[r][cg * 8 + e] = mx[e];
   }
   __syncthreads();
+  a = FLT_MAX;
+  b = -FLT_MAX;
   if (threadIdx.x < kD) {
-    float a = FLT_MAX, b = -FLT_MAX;
     for (int q = 0; q < kRpi; ++q) {
       a = fminf(a, smn[q][threadIdx.x]);
       b = fmaxf(b, smx[q][threadIdx.x]);
     }
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_stats(const T* __restrict__ x, int n, int S,
+                                                    float* __restrict__ part) {
+  const int row = blockIdx.x, s = blockIdx.y;
+  const int per = (n + S - 1) / S;
+  const int i0 = s * per, i1 = min(n, i0 + per);
+  float a, b;
+  tile_minmax<T>(x + (size_t)row * n * kD, i0, i1, a, b);
+  if (threadIdx.x < kD) {
     float* out = part + ((size_t)row * S + s) * 2 * kD;
     out[threadIdx.x] = a;
     out[kD + threadIdx.x] = b;
   }
 }
 
-// Folds the S partials of `row` into shared alpha/beta/inv; block (row, 0)
-// also writes the stored alpha and step.
+// Folds the S partials of `row` ([S][min, max][kD], global or shared memory)
+// into shared alpha/beta/inv; with `write` also stores the row's alpha and step.
 template <typename T>
-__device__ __forceinline__ void fold_stats(const float* __restrict__ part, int row, int S, int L,
+__device__ __forceinline__ void fold_stats(const float* p, int S, int L, bool write, int row,
                                            float* s_alpha, float* s_beta, float* s_inv,
                                            T* __restrict__ alpha_out, T* __restrict__ scale_out) {
   if (threadIdx.x < kD) {
     const int j = threadIdx.x;
     float a = FLT_MAX, b = -FLT_MAX;
-    const float* p = part + (size_t)row * S * 2 * kD;
     for (int s = 0; s < S; ++s) {
       a = fminf(a, p[s * 2 * kD + j]);
       b = fmaxf(b, p[s * 2 * kD + kD + j]);
@@ -78,7 +90,7 @@ __device__ __forceinline__ void fold_stats(const float* __restrict__ part, int r
     s_alpha[j] = a;
     s_beta[j] = b;
     s_inv[j] = (b > a) ? (float)L / (b - a) : 0.f;
-    if (blockIdx.y == 0) {
+    if (write) {
       alpha_out[(size_t)row * kD + j] = DT<T>::from_float(a);  // exact: an input value
       const double step = __ddiv_rn(__dsub_rn((double)b, (double)a), (double)L);
       scale_out[(size_t)row * kD + j] = DT<T>::from_double(step);
@@ -89,13 +101,9 @@ __device__ __forceinline__ void fold_stats(const float* __restrict__ part, int r
 
 // Canonical layout: each thread turns 8 channels of one token into 8*BITS bits.
 template <typename T, int BITS>
-__global__ void __launch_bounds__(kThreads) k_pack_canonical(
-    const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
-    uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
+__device__ __forceinline__ void k_pack_canonical_tile(const T* __restrict__ x, int n, int row, int tile, int tile_tokens,
+    const float* s_alpha, const float* s_beta, const float* s_inv, uint8_t* __restrict__ codes) {
   constexpr int L = (1 << BITS) - 1;
-  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
-  const int row = blockIdx.x;
-  fold_stats<T>(part, row, S, L, s_alpha, s_beta, s_inv, alpha_out, scale_out);
   const int cg = threadIdx.x % kTpr, r = threadIdx.x / kTpr;
   float af[8], inv[8], hi[8], lo[8];
   double ad[8], bd[8];
@@ -107,7 +115,7 @@ __global__ void __launch_bounds__(kThreads) k_pack_canonical(
     bd[e] = (double)s_beta[cg * 8 + e];
     two_sum(af[e], s_beta[cg * 8 + e], hi[e], lo[e]);  // used for 1-bit codes
   }
-  const int i0 = blockIdx.y * tile_tokens, i1 = min(n, i0 + tile_tokens);
+  const int i0 = tile * tile_tokens, i1 = min(n, i0 + tile_tokens);
   const T* xr = x + (size_t)row * n * kD + cg * 8;
   uint8_t* cr = codes + (size_t)row * n * (kD * BITS / 8) + cg * BITS;
   for (int i = i0 + r; i < i1; i += kRpi) {
@@ -129,21 +137,28 @@ __global__ void __launch_bounds__(kThreads) k_pack_canonical(
   }
 }
 
-// OCTET_K layout (bits = 1): a thread owns one token octet (8 tokens) x 8
-// channels, i.e. 8 consecutive bytes of the layout.
-template <typename T>
-__global__ void __launch_bounds__(kThreads) k_pack_octet_k(
+template <typename T, int BITS>
+__global__ void __launch_bounds__(kThreads) k_pack_canonical(
     const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
     uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
   __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
   const int row = blockIdx.x;
-  fold_stats<T>(part, row, S, 1, s_alpha, s_beta, s_inv, alpha_out, scale_out);
+  fold_stats<T>(part + (size_t)row * S * 2 * kD, S, (1 << BITS) - 1, blockIdx.y == 0, row, s_alpha, s_beta, s_inv, alpha_out,
+                scale_out);
+  k_pack_canonical_tile<T, BITS>(x, n, row, blockIdx.y, tile_tokens, s_alpha, s_beta, s_inv, codes);
+}
+
+// OCTET_K layout (bits = 1): a thread owns one token octet (8 tokens) x 8
+// channels, i.e. 8 consecutive bytes of the layout.
+template <typename T>
+__device__ __forceinline__ void k_pack_octet_k_tile(const T* __restrict__ x, int n, int row, int tile, int tile_tokens,
+    const float* s_alpha, const float* s_beta, const float* s_inv, uint8_t* __restrict__ codes) {
   const int cb = threadIdx.x % kTpr, r = threadIdx.x / kTpr;
   float hi[8], lo[8];  // alpha + beta of the thread's channels as an exact pair
 #pragma unroll
   for (int e = 0; e < 8; ++e) two_sum(s_alpha[cb * 8 + e], s_beta[cb * 8 + e], hi[e], lo[e]);
   const int octets = (n + 7) / 8;
-  const int m0 = blockIdx.y * (tile_tokens / 8), m1 = min(octets, m0 + tile_tokens / 8);
+  const int m0 = tile * (tile_tokens / 8), m1 = min(octets, m0 + tile_tokens / 8);
   const T* xr = x + (size_t)row * n * kD + cb * 8;
   uint8_t* cr = codes + (size_t)row * octets * kD + cb * 8;
   for (int m = m0 + r; m < m1; m += kRpi) {
@@ -163,58 +178,81 @@ __global__ void __launch_bounds__(kThreads) k_pack_octet_k(
   }
 }
 
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_pack_octet_k(
+    const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
+    uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
+  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
+  const int row = blockIdx.x;
+  fold_stats<T>(part + (size_t)row * S * 2 * kD, S, 1, blockIdx.y == 0, row, s_alpha, s_beta, s_inv, alpha_out,
+                scale_out);
+  k_pack_octet_k_tile<T>(x, n, row, blockIdx.y, tile_tokens, s_alpha, s_beta, s_inv, codes);
+}
+
 // OCTET_V layout (bits = 1): a warp owns 32 consecutive tokens; lane l reads
 // token l's row and the warp ballots each channel into one 32-token word,
 // which is bytes 4q..4q+3 of that channel's 32-byte row in the 256-token tile.
+template <typename T>
+__device__ __forceinline__ void k_pack_octet_v_tile(const T* __restrict__ x, int n, int row, int tile, int tile_tokens,
+    const float* s_alpha, const float* s_beta, const float* s_inv, uint8_t* __restrict__ codes) {
+  __shared__ float s_hi[kD], s_lo[kD];  // alpha + beta per channel as an exact pair
+  if (threadIdx.x < kD) two_sum(s_alpha[threadIdx.x], s_beta[threadIdx.x], s_hi[threadIdx.x], s_lo[threadIdx.x]);
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n_pad = (n + 255) / 256 * 256;
+  const int b0 = tile * (tile_tokens / 32), b1 = min(n_pad / 32, b0 + tile_tokens / 32);
+  const T* xr = x + (size_t)row * n * kD;
+  uint8_t* cr = codes + (size_t)row * (n_pad / 256) * 4096;
+  // Every warp runs every pass (the trip count depends on the tile only): a
+  // ballot inside a loop whose trip count the compiler sees as per-thread costs
+  // several times its latency. A pass past the tile's end ballots zeros and
+  // stores nothing.
+  const int warp_u = __shfl_sync(0xffffffffu, warp, 0);
+  for (int pass = 0; pass < b1 - b0; pass += kThreads / 32) {
+    const int blk = b0 + pass + warp_u;
+    const int i = blk * 32 + lane;
+    const bool live = blk < b1 && i < n;
+    uint32_t words[4] = {0, 0, 0, 0};  // channels lane, lane+32, lane+64, lane+96
+#pragma unroll 4
+    for (int cg = 0; cg < kD / 8; ++cg) {
+      float v[8];
+      if (live) load8(xr + (size_t)i * kD + cg * 8, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int j = cg * 8 + e;
+        const uint32_t code = live ? code1(v[e], s_hi[j], s_lo[j]) : 0u;
+        const uint32_t bal = __ballot_sync(0xffffffffu, code);
+        if ((j & 31) == lane) words[j >> 5] = bal;
+      }
+    }
+    if (blk < b1) {
+      const int vt = blk >> 3, q = blk & 7;  // 256-token tile of the layout, word within its 32-byte row
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int j = w * 32 + lane;
+        *reinterpret_cast<uint32_t*>(cr + (size_t)vt * 4096 + j * 32 + q * 4) = words[w];
+      }
+    }
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_pack_octet_v(
     const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
     uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
   __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
   const int row = blockIdx.x;
-  fold_stats<T>(part, row, S, 1, s_alpha, s_beta, s_inv, alpha_out, scale_out);
-  __shared__ float s_hi[kD], s_lo[kD];  // alpha + beta per channel as an exact pair
-  if (threadIdx.x < kD) two_sum(s_alpha[threadIdx.x], s_beta[threadIdx.x], s_hi[threadIdx.x], s_lo[threadIdx.x]);
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int n_pad = (n + 255) / 256 * 256;
-  const int b0 = blockIdx.y * (tile_tokens / 32), b1 = min(n_pad / 32, b0 + tile_tokens / 32);
-  const T* xr = x + (size_t)row * n * kD;
-  uint8_t* cr = codes + (size_t)row * (n_pad / 256) * 4096;
-  for (int blk = b0 + warp; blk < b1; blk += kThreads / 32) {
-    const int i = blk * 32 + lane;
-    uint32_t words[4] = {0, 0, 0, 0};  // channels lane, lane+32, lane+64, lane+96
-#pragma unroll 4
-    for (int cg = 0; cg < kD / 8; ++cg) {
-      float v[8];
-      if (i < n) load8(xr + (size_t)i * kD + cg * 8, v);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int j = cg * 8 + e;
-        const uint32_t code = (i < n) ? code1(v[e], s_hi[j], s_lo[j]) : 0u;
-        const uint32_t bal = __ballot_sync(0xffffffffu, code);
-        if ((j & 31) == lane) words[j >> 5] = bal;
-      }
-    }
-    const int tile = blk >> 3, q = blk & 7;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const int j = w * 32 + lane;
-      *reinterpret_cast<uint32_t*>(cr + (size_t)tile * 4096 + j * 32 + q * 4) = words[w];
-    }
-  }
+  fold_stats<T>(part + (size_t)row * S * 2 * kD, S, 1, blockIdx.y == 0, row, s_alpha, s_beta, s_inv, alpha_out,
+                scale_out);
+  k_pack_octet_v_tile<T>(x, n, row, blockIdx.y, tile_tokens, s_alpha, s_beta, s_inv, codes);
 }
 
 // OCTET_K layout with BITS in {2, 4, 8}: P = 8 / BITS tokens share a byte; a
 // thread owns one byte group (P tokens) x 8 channels, i.e. 8 consecutive bytes.
 template <typename T, int BITS>
-__global__ void __launch_bounds__(kThreads) k_pack_octet_k_b(
-    const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
-    uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
+__device__ __forceinline__ void k_pack_octet_k_b_tile(const T* __restrict__ x, int n, int row, int tile, int tile_tokens,
+    const float* s_alpha, const float* s_beta, const float* s_inv, uint8_t* __restrict__ codes) {
   constexpr int L = (1 << BITS) - 1, P = 8 / BITS;
-  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
-  const int row = blockIdx.x;
-  fold_stats<T>(part, row, S, L, s_alpha, s_beta, s_inv, alpha_out, scale_out);
   const int cb = threadIdx.x % kTpr, r = threadIdx.x / kTpr;
   float af[8], inv[8];
   double ad[8], bd[8];
@@ -226,7 +264,7 @@ __global__ void __launch_bounds__(kThreads) k_pack_octet_k_b(
     bd[e] = (double)s_beta[cb * 8 + e];
   }
   const int groups = (n + P - 1) / P;
-  const int m0 = blockIdx.y * (tile_tokens / P), m1 = min(groups, m0 + tile_tokens / P);
+  const int m0 = tile * (tile_tokens / P), m1 = min(groups, m0 + tile_tokens / P);
   const T* xr = x + (size_t)row * n * kD + cb * 8;
   uint8_t* cr = codes + (size_t)row * groups * kD + cb * 8;
   for (int m = m0 + r; m < m1; m += kRpi) {
@@ -246,20 +284,27 @@ __global__ void __launch_bounds__(kThreads) k_pack_octet_k_b(
   }
 }
 
+template <typename T, int BITS>
+__global__ void __launch_bounds__(kThreads) k_pack_octet_k_b(
+    const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
+    uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
+  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
+  const int row = blockIdx.x;
+  fold_stats<T>(part + (size_t)row * S * 2 * kD, S, (1 << BITS) - 1, blockIdx.y == 0, row, s_alpha, s_beta, s_inv, alpha_out,
+                scale_out);
+  k_pack_octet_k_b_tile<T, BITS>(x, n, row, blockIdx.y, tile_tokens, s_alpha, s_beta, s_inv, codes);
+}
+
 // OCTET_V layout with BITS in {2, 4, 8}: tiles of 32 P tokens; byte column q of
 // a tile holds tokens P q .. P q + P - 1. A warp owns one tile: lane q builds
 // byte column q of every channel (consecutive lanes write consecutive bytes).
 template <typename T, int BITS>
-__global__ void __launch_bounds__(kThreads) k_pack_octet_v_b(
-    const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
-    uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
+__device__ __forceinline__ void k_pack_octet_v_b_tile(const T* __restrict__ x, int n, int row, int tile, int tile_tokens,
+    const float* s_alpha, const float* s_beta, const float* s_inv, uint8_t* __restrict__ codes) {
   constexpr int L = (1 << BITS) - 1, P = 8 / BITS, kTile = 32 * P;
-  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
-  const int row = blockIdx.x;
-  fold_stats<T>(part, row, S, L, s_alpha, s_beta, s_inv, alpha_out, scale_out);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int tiles = (n + kTile - 1) / kTile;
-  const int v0 = blockIdx.y * (tile_tokens / kTile), v1 = min(tiles, v0 + tile_tokens / kTile);
+  const int v0 = tile * (tile_tokens / kTile), v1 = min(tiles, v0 + tile_tokens / kTile);
   const T* xr = x + (size_t)row * n * kD;
   uint8_t* cr = codes + (size_t)row * tiles * 4096;
   for (int vt = v0 + warp; vt < v1; vt += kThreads / 32) {
@@ -286,6 +331,112 @@ __global__ void __launch_bounds__(kThreads) k_pack_octet_v_b(
   }
 }
 
+template <typename T, int BITS>
+__global__ void __launch_bounds__(kThreads) k_pack_octet_v_b(
+    const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
+    uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
+  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
+  const int row = blockIdx.x;
+  fold_stats<T>(part + (size_t)row * S * 2 * kD, S, (1 << BITS) - 1, blockIdx.y == 0, row, s_alpha, s_beta, s_inv, alpha_out,
+                scale_out);
+  k_pack_octet_v_b_tile<T, BITS>(x, n, row, blockIdx.y, tile_tokens, s_alpha, s_beta, s_inv, codes);
+}
+
+// Single-read fill: one thread-block cluster per row, one CTA per tile of
+// kFillTile tokens. Each CTA takes the min / max of its tile, pushes them to
+// every CTA of the cluster (distributed shared memory), folds the row's
+// statistics from what it received (the same fold as the two-launch path, so
+// alpha, step and codes are identical) and packs its own tile. The pack re-reads
+// the tile the CTA has just read: the launcher caps the CTAs resident per SM so
+// that the tiles in flight stay well inside L2, and HBM sees the input once.
+constexpr int kFillMaxCl = 16;
+
+template <typename T, int BITS, int LAYOUT>
+__global__ void __launch_bounds__(kThreads, 4) k_fill(const T* __restrict__ x, int n, int cl, int tile_tokens,
+                                                   uint8_t* __restrict__ codes, T* __restrict__ alpha_out,
+                                                   T* __restrict__ scale_out) {
+  __shared__ float recv[kFillMaxCl][2][kD];  // every CTA's (min, max) per channel
+  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
+  const uint32_t rank = tc::cluster_rank();
+  const int row = blockIdx.x / cl;
+  tc::cluster_arrive_relaxed();  // matched by the wait before the first peer store
+  const int i0 = (int)rank * tile_tokens, i1 = min(n, i0 + tile_tokens);
+  float a, b;
+  tile_minmax<T>(x + (size_t)row * n * kD, i0, i1, a, b);
+  tc::cluster_wait();  // every CTA of the cluster is running
+  if (threadIdx.x < kD) {
+    for (int r = 0; r < cl; ++r) {
+      tc::st_peer_f32(&recv[rank][0][threadIdx.x], (uint32_t)r, a);
+      tc::st_peer_f32(&recv[rank][1][threadIdx.x], (uint32_t)r, b);
+    }
+  }
+  tc::cluster_sync();  // every partial has landed; no peer access after this point
+  constexpr int L = (1 << BITS) - 1;
+  fold_stats<T>(&recv[0][0][0], cl, L, rank == 0, row, s_alpha, s_beta, s_inv, alpha_out, scale_out);
+  const int tile = (int)rank;
+  if constexpr (LAYOUT == CQ_LAYOUT_CANONICAL) {
+    k_pack_canonical_tile<T, BITS>(x, n, row, tile, tile_tokens, s_alpha, s_beta, s_inv, codes);
+  } else if constexpr (LAYOUT == CQ_LAYOUT_OCTET_K) {
+    if constexpr (BITS == 1)
+      k_pack_octet_k_tile<T>(x, n, row, tile, tile_tokens, s_alpha, s_beta, s_inv, codes);
+    else
+      k_pack_octet_k_b_tile<T, BITS>(x, n, row, tile, tile_tokens, s_alpha, s_beta, s_inv, codes);
+  } else {
+    if constexpr (BITS == 1)
+      k_pack_octet_v_tile<T>(x, n, row, tile, tile_tokens, s_alpha, s_beta, s_inv, codes);
+    else
+      k_pack_octet_v_b_tile<T, BITS>(x, n, row, tile, tile_tokens, s_alpha, s_beta, s_inv, codes);
+  }
+}
+
+// Tile of the single-read fill for a row of n tokens (0: not supported, use
+// the two-launch path): 512 tokens up to n = 8192, 1024 up to n = 16384.
+int fill_tile_tokens(int n) {
+  if (n <= 512 * kFillMaxCl) return 512;
+  if (n <= 1024 * kFillMaxCl) return 1024;
+  return 0;
+}
+
+template <typename T, int BITS, int LAYOUT>
+cudaError_t launch_fill(const T* x, int rows, int n, uint8_t* codes, T* alpha, T* scale, cudaStream_t stream) {
+  const int tile = fill_tile_tokens(n);
+  const int cl = (n + tile - 1) / tile;
+  // Dynamic shared memory only to cap residency at 4 CTAs per SM: 4 x 148 tiles
+  // of 512 tokens x 256 B = 76 MB in flight, inside the 126 MB L2, so each
+  // tile's second read hits L2 (at 1024-token tiles the cap is the same).
+  constexpr int kPad = 12 * 1024;
+  static bool attr_set = false;  // benign race: every caller sets the same values
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_fill<T, BITS, LAYOUT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(rows * cl), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kPad;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_fill<T, BITS, LAYOUT>, x, n, cl, tile, codes, alpha, scale);
+}
+
+template <typename T, int LAYOUT>
+cudaError_t launch_fill_bits(const T* x, int rows, int n, int bits, uint8_t* codes, T* alpha, T* scale,
+                             cudaStream_t stream) {
+  switch (bits) {
+    case 1: return launch_fill<T, 1, LAYOUT>(x, rows, n, codes, alpha, scale, stream);
+    case 2: return launch_fill<T, 2, LAYOUT>(x, rows, n, codes, alpha, scale, stream);
+    case 4: return launch_fill<T, 4, LAYOUT>(x, rows, n, codes, alpha, scale, stream);
+    default: return launch_fill<T, 8, LAYOUT>(x, rows, n, codes, alpha, scale, stream);
+  }
+}
+
 }  // namespace
 
 int quantize_splits(int rows, int n) {
@@ -301,6 +452,16 @@ template <typename T>
 static cudaError_t launch_quantize_t(const T* x, int rows, int n, int bits, cq_layout layout,
                                      uint8_t* codes, T* alpha, T* scale, float* part,
                                      cudaStream_t stream) {
+  if (fill_tile_tokens(n) > 0 && (long long)rows * ((n + fill_tile_tokens(n) - 1) / fill_tile_tokens(n)) <= 0x7fffffffLL) {
+    cudaError_t e;
+    if (layout == CQ_LAYOUT_CANONICAL)
+      e = launch_fill_bits<T, CQ_LAYOUT_CANONICAL>(x, rows, n, bits, codes, alpha, scale, stream);
+    else if (layout == CQ_LAYOUT_OCTET_K)
+      e = launch_fill_bits<T, CQ_LAYOUT_OCTET_K>(x, rows, n, bits, codes, alpha, scale, stream);
+    else
+      e = launch_fill_bits<T, CQ_LAYOUT_OCTET_V>(x, rows, n, bits, codes, alpha, scale, stream);
+    return e == cudaSuccess ? cudaGetLastError() : e;
+  }
   const int S = quantize_splits(rows, n);
   k_stats<T><<<dim3(rows, S), kThreads, 0, stream>>>(x, n, S, part);
   const int tile = 1024;

@@ -132,7 +132,12 @@ cq_status cq_quantize_kv_workspace_size(int B, int H, int n, int d, size_t* byte
  * (x - alpha_j) * L / (beta_j - alpha_j), L = 2^bits - 1, ties to even, taken
  * on the IEEE double evaluation ((x - alpha) * L) / (beta - alpha); 0 when
  * beta_j == alpha_j. (For binary16 inputs this is the exact real rounding.)
- * The octet layouts require bits = 1.
+ * The octet layouts take bits in {1, 2, 4, 8} with d = 128.
+ *
+ * Execution: for n <= 16384 one launch reads x once (a thread-block cluster
+ * per (b, h) row exchanges the channel statistics on chip, and each CTA packs
+ * the tile it has just read); longer rows take two launches (statistics into
+ * the workspace, then pack). Both give identical alpha, scale and codes.
  */
 cq_status cq_quantize_kv(const void* x, cq_dtype dt, int B, int H, int n, int d, int bits,
                          cq_layout layout, uint8_t* codes, void* alpha, void* scale,
