@@ -61,3 +61,23 @@ def test_mixed_without_text_equals_plain_decode(cuda_device, bits):
     mixed = cq.cq_decode_attn_mixed(qd, kq, vq, None, None, calib=(True, 0.8, 0.9))
     torch.cuda.synchronize()
     assert torch.equal(plain, mixed)
+
+
+def test_mixed_through_the_row_kernel(cuda_device):
+    """Enough (sequence, kv-head) rows for the one-CTA-per-row kernel (partial
+    mode), then the text merge; and equality with the plain decode without text."""
+    B, Hkv = 38, 4  # 152 rows: at least one per SM
+    if cq.cq_decode_kernel_name(cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V, B, 4 * Hkv, Hkv, 700, 128, 1) != "k_decode_row":
+        pytest.skip("this device has more SMs than rows: the row kernel is not chosen")
+    q, k, v, kt, vt = _case(B, Hkv, 700, 50, "f16", 1, seed=77)
+    qd = q.to(cuda_device)
+    kq = cq.cq_quantize_kv(k.to(cuda_device), 1, cq.LAYOUT_OCTET_K)
+    vq = cq.cq_quantize_kv(v.to(cuda_device), 1, cq.LAYOUT_OCTET_V)
+    calib = (True, 0.8, 0.9)
+    out = cq.cq_decode_attn_mixed(qd, kq, vq, kt.to(cuda_device), vt.to(cuda_device), calib=calib)
+    plain = cq.cq_decode_attn(qd, kq, vq, calib=calib)
+    mixed0 = cq.cq_decode_attn_mixed(qd, kq, vq, None, None, calib=calib)
+    torch.cuda.synchronize()
+    ref = oracle.decode_attention_mixed(f64(q), f64(k), f64(v), f64(kt), f64(vt), 1, "f16", calib)["out"]
+    assert row_rel_err(out.float().cpu().numpy(), ref_output_rounded(ref, torch.float16)) <= OUT_RTOL
+    assert torch.equal(plain, mixed0)
