@@ -37,12 +37,15 @@
 //     bit pair in its own tensor-memory lane;
 //  4. the row range per head (warp shuffles + one CTA barrier) gives the
 //     calibration slope;
-//  5. V side: warp pair (q, q + 4) takes tiles q, q + 4, ... and splits the 128
-//     channels. Per tile a lane reads back its 32 logits, forms P = p 2^(31-k)
-//     for its bit of every pair, swaps them with lane ^ 16 and assembles the A
-//     fragment (rows 4 limb + head, columns octets) with byte permutes;
-//     B = V codes of 8 channels masked to bit k. Sum_l 2^(8l-31) D_l = sum c p;
-//  6. the four warp pairs' sums meet in shared memory; o = alpha_V + s_V (.)
+//  5. each lane turns its 32 logit columns of a tile, in place, into its A-fragment
+//     words of the tile's 8 bit positions for the V side: P = p 2^(31-k) for its
+//     own bit of every pair, a swap with lane ^ 16, byte permutes into limb rows
+//     (rows 4 limb + head, columns octets);
+//  6. V side: warp pair (q, q + 4) (the two warps sharing a tensor-memory lane
+//     quarter) takes tiles q, q + 4, ... and splits the 128 channels; A = the
+//     tile's fragments loaded from tensor memory, B = V codes of 8 channels
+//     masked to bit k. Sum_l 2^(8l-31) D_l = sum c p;
+//  7. the four warp pairs' sums meet in shared memory; o = alpha_V + s_V (.)
 //     sum c p / sum p.
 // One launch per decode step, no workspace; n <= 8192 tokens per row.
 #include <float.h>
@@ -80,12 +83,8 @@ struct RowFixed {
   float red[8][kG][2];             // per-warp reduction scratch
   float lsum[8][kG];               // per warp: sum of its softmax weights
   float c0[kG], kscale[kG], alog2[kG], ref[kG], cst[kG];
-  // V-side A fragments of one tile, per warp pair, double-buffered by tile:
-  // [pair][buffer][bit][lane][4 words]; afterwards the pairs' partial sums
-  // [pair][head][channel] (fp32) reuse the space
-  alignas(16) uint32_t frag[4][2][8][32][4];
+  alignas(16) float part[4][kG][kD];  // per warp pair: sum_i c_ij p_i
 };
-static_assert(sizeof(float) * 4 * kG * kD <= sizeof(uint32_t) * 4 * 2 * 8 * 32 * 4, "partial sums fit");
 
 __host__ __device__ constexpr size_t row_smem_bytes() {
   return (size_t)kSlots * kChunkBytes + sizeof(RowFixed) + 1024;  // + alignment to the swizzle atom
@@ -366,23 +365,78 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     __syncthreads();
 
-    // ---- 5. V side: pair q = warp & 3 takes tiles q, q + 4, ...; hc = warp >> 2 picks
-    // channels 64 hc .. 64 hc + 63 and forms the weight fragments of bits 4 hc .. 4 hc + 3
+    // ---- 5. softmax weights, as the V side's A fragments, in tensor memory. A
+    // lane's 32 logit columns of a tile become, in place, its A-fragment words of
+    // the tile's 8 bit positions (column 4 k + r = register r of bit k): P =
+    // p 2^(31-k) for its own bit of every pair, a swap with lane ^ 16 (the lane
+    // holding the same head's other limbs), byte permutes into limb rows. Warp w
+    // takes the tiles it wrote on the K side; every warp runs every pass (uniform
+    // trip count), a pass past the last chunk loads and stores nothing.
     const int q = warp & 3, hc = warp >> 2;
-    const float alog2 = F.alog2[h], ref = F.ref[h];
-    const uint32_t sel = lo ? 0x6240u : 0x7351u;  // bytes (limb, limb + 2) of two words: limbs 0, 2 or 1, 3
-    const uint32_t frag_u = tc::smem_u32(&F.frag[q][0][0][0][0]) + (uint32_t)lane * 16;
+    float lsum = 0.f;
+    {
+      const float alog2 = F.alog2[h], ref = F.ref[h];
+      const uint32_t sel = lo ? 0x6240u : 0x7351u;  // bytes (limb, limb + 2) of two words: limbs 0, 2 or 1, 3
+      for (int pass = 0; pass < nchunk; pass += 2) {
+        const int jj = pass + hc, j = kChunkTiles * jj + q;  // chunk and tile
+        const bool act = jj < nchunk;
+        const bool ragged = kTile * (j + 1) > n;  // true for a tile past the row's end: every token masked
+        const uint32_t col = tlane + (uint32_t)(32 * jj);
+        uint32_t xs[32], outw[32];
+        if (act) {
+          tc::ld_x16(col, *reinterpret_cast<uint32_t(*)[16]>(&xs[0]));
+          tc::ld_x16(col + 16, *reinterpret_cast<uint32_t(*)[16]>(&xs[16]));
+          tc::wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) xs[i] = 0u;
+        }
+#pragma unroll
+        for (int kp = 0; kp < 4; ++kp) {
+          const int kown = 2 * kp + (lo ? 0 : 1);
+          const float bias = (float)(31 - kown) - ref;
+          const float unscale = __int_as_float((127 - 31 + kown) << 23);  // 2^(k - 31)
+          uint32_t pown[8], poth[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float p = ex2_approx(fmaf(__uint_as_float(xs[8 * kp + i]), alog2, bias));
+            const bool ok = act && (!ragged || kTile * j + 8 * lane_octet(tq, i) + kown < n);
+            pown[i] = ok ? __float2uint_rn(p) : 0u;
+            lsum = ok ? fmaf(p, unscale, lsum) : lsum;
+            poth[i] = __shfl_xor_sync(0xffffffffu, pown[i], 16);
+          }
+          // bit 2 kp: the lo lanes' weights; bit 2 kp + 1: the hi lanes'
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            uint32_t P[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) P[i] = ((kk == 0) == lo) ? pown[i] : poth[i];
+            const int b = 4 * (2 * kp + kk);
+            gather_limbs(P[0], P[1], P[2], P[3], sel, outw[b], outw[b + 1]);
+            gather_limbs(P[4], P[5], P[6], P[7], sel, outw[b + 2], outw[b + 3]);
+          }
+        }
+        if (act) {
+          tc::st_x32(col, outw);
+        }
+      }
+      tc::wait_st();
+    }
+    tc::fence_before_sync();
+    __syncthreads();  // the other warp of each pair reads these fragments
+    tc::fence_after_sync();
+
+    // ---- 6. V side: warp pair (q, q + 4) takes tiles q, q + 4, ...; hc picks
+    // channels 64 hc .. 64 hc + 63. A = the tile's fragments from tensor memory,
+    // B = V codes of 8 channels masked to bit k.
     int acc[8][4];
 #pragma unroll
     for (int jn = 0; jn < 8; ++jn) acc[jn][0] = acc[jn][1] = acc[jn][2] = acc[jn][3] = 0;
-    float lsum = 0.f;
-    int buf = 0;
     for (int c = 0; c < nchunk; ++c) {
       const int gi = nchunk + c, s = gi % kSlots, j = kChunkTiles * c + q;
       warp_wait_copies(&F.full[s], (uint32_t)(gi / kSlots) & 1u, err);
       uint32_t bv[8][2];
-      const bool have = j < nt;
-      if (have) {
+      if (j < nt) {
         const uint32_t tile_u = ring_u + (uint32_t)(s * kChunkBytes + q * 4096);
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
@@ -400,57 +454,25 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int jn = 0; jn < 8; ++jn) bv[jn][0] = bv[jn][1] = 0u;
       }
       release_chunk(F, ring, &kmap, &vmap, row, nchunk, gi, 1);  // V side: all eight warps per chunk
-      // no skip for a missing tile (zero codes, zero weights): the shuffles below
-      // stay out of branches on the warp index
-      const bool ragged = kTile * (j + 1) > n;  // true for a missing tile: every token masked
-      uint32_t xs[16];  // logits of bit pairs 2 hc, 2 hc + 1 (this lane's bit of each)
-      tc::ld_x16(tlane + (uint32_t)(32 * (j >> 2) + 16 * hc), xs);
+      uint32_t fr[32];  // A fragments of the tile's 8 bit positions (zero past the row's end)
+      tc::ld_x16(tlane + (uint32_t)(32 * c), *reinterpret_cast<uint32_t(*)[16]>(&fr[0]));
+      tc::ld_x16(tlane + (uint32_t)(32 * c + 16), *reinterpret_cast<uint32_t(*)[16]>(&fr[16]));
       tc::wait_ld();
-      const uint32_t fbuf = frag_u + (uint32_t)buf * 4096;
-#pragma unroll
-      for (int kq = 0; kq < 2; ++kq) {
-        const int kp = 2 * hc + kq, kown = 2 * kp + (lo ? 0 : 1);
-        const float bias = (float)(31 - kown) - ref;
-        const float unscale = __int_as_float((127 - 31 + kown) << 23);  // 2^(k - 31)
-        uint32_t pown[8], poth[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float p = ex2_approx(fmaf(__uint_as_float(xs[8 * kq + i]), alog2, bias));
-          const bool ok = !ragged || kTile * j + 8 * lane_octet(tq, i) + kown < n;
-          pown[i] = ok ? __float2uint_rn(p) : 0u;
-          lsum = ok ? fmaf(p, unscale, lsum) : lsum;
-          poth[i] = __shfl_xor_sync(0xffffffffu, pown[i], 16);
-        }
-        // bit 2 kp: the lo lanes' weights; bit 2 kp + 1: the hi lanes'
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          uint32_t P[8], af[4];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) P[i] = ((kk == 0) == lo) ? pown[i] : poth[i];
-          gather_limbs(P[0], P[1], P[2], P[3], sel, af[0], af[1]);
-          gather_limbs(P[4], P[5], P[6], P[7], sel, af[2], af[3]);
-          sts128(fbuf + (uint32_t)(2 * kp + kk) * 512, af);
-        }
-      }
-      tc::bar_sync(2 + q, 64);  // the pair's weight fragments of this tile are complete
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        uint32_t af[4];
-        lds128(fbuf + (uint32_t)k * 512, af);
+        const uint32_t af[4] = {fr[4 * k], fr[4 * k + 1], fr[4 * k + 2], fr[4 * k + 3]};
         const uint32_t msk = 0x01010101u << k;
 #pragma unroll
         for (int jn = 0; jn < 8; ++jn) mma_u8u8(acc[jn], af, bv[jn][0] & msk, bv[jn][1] & msk);
       }
-      buf ^= 1;
     }
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
     if (lo && tq == 0) F.lsum[warp][g] = lsum;
 
-    // ---- 6. limbs combined (lane and lane ^ 16), the pairs summed, o written
-    __syncthreads();  // every warp is done with the fragment buffers: the partial sums reuse them
-    float* part = reinterpret_cast<float*>(&F.frag[0][0][0][0][0]);  // [pair][head][channel]
+    // ---- 7. limbs combined (lane and lane ^ 16), the pairs summed, o written
+    float* part = &F.part[0][0][0];  // [pair][head][channel]
     {
       const float s_lo = lo ? 0x1p-31f : 0x1p-23f, s_hi = lo ? 0x1p-15f : 0x1p-7f;
 #pragma unroll
