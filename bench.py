@@ -386,6 +386,62 @@ def cpu_baseline(w):
                       f"quantized cache; {secs:.1f} s"}
 
 
+def _oracle_timed_task(task):
+    """One worker of the all-cores oracle baseline: builds its inputs, waits for
+    the common start time, then decodes whole rows until the common end time;
+    returns the rows it finished in the window."""
+    wname, seed, start, span = task
+    from oracle import calibquant as oc
+    import oracle
+    w = synth.WORKLOADS[wname]
+    q, k, v = synth.make_case(1, 4, 1, w.n, w.d, w.dtype, w.outliers, seed, "cpu")
+    f = lambda t: t.to(torch.float64).numpy()
+    q, k, v = f(q), f(k), f(v)
+    kq = oracle.quantize_cache(k, 1, w.dtype)
+    vq = oracle.quantize_cache(v, 1, w.dtype)
+    rows = 0
+    with threadpool_limits(limits=1):
+        while time.time() < start:
+            time.sleep(0.01)
+        while time.time() < start + span:
+            _oracle_rows(oc, q, kq, vq, 1)
+            rows += 1
+    return rows
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline_all_cores(w, wname: str, span: float = 10.0):
+    """The oracle on every host core at once (one single-threaded process per
+    core, at most 32): rows finished by all processes in a common window."""
+    import multiprocessing as mp
+    from concurrent.futures import ProcessPoolExecutor
+    nproc = os.cpu_count() or 1
+    workers = max(1, min(nproc, 32))
+    start = time.time() + 45.0  # spawn, imports and inputs finish before the window opens
+    try:  # a worker that dies raises here instead of leaving the bench waiting
+        with ProcessPoolExecutor(workers, mp_context=mp.get_context("spawn")) as ex:
+            futs = [ex.submit(_oracle_timed_task, (wname, 500 + i, start, span)) for i in range(workers)]
+            rows = sum(f.result(timeout=120 + span) for f in futs)
+    except Exception as e:  # noqa: BLE001 -- a baseline, reported as missing rather than failing the bench
+        return {"value": None, "unit": "tokens/s", "cores": workers, "nproc": nproc, "kind": "oracle",
+                "error": f"{type(e).__name__}: {e}"[:200]}
+    seqs = rows / w.hkv
+    return {"value": seqs / span, "unit": "tokens/s", "cores": workers, "nproc": nproc, "cpu_model": cpu_model(),
+            "kind": "oracle",
+            "sample": f"{rows} (sequence, kv-head) rows of {wname} decoded by {workers} single-threaded "
+                      f"processes in a common {span:.0f} s window (fp64 numpy)"}
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return None
@@ -542,6 +598,9 @@ def main():
         line = run_ours(args, world, rank, local)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(synth.WORKLOADS[args.workload])
+            line["cpu_baseline"]["nproc"] = os.cpu_count() or 1
+            line["cpu_baseline"]["cpu_model"] = cpu_model()
+            line["cpu_baseline_all_cores"] = cpu_baseline_all_cores(synth.WORKLOADS[args.workload], args.workload)
     if rank == 0 and line is not None:
         print(json.dumps(line), flush=True)
     if world > 1:
