@@ -20,23 +20,37 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kG = 4;
 
-// Four consecutive elements of a row as floats.
-__device__ __forceinline__ void load4(const half* p, float (&v)[4]) {
-  const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
-  const float2 a = __half22float2(*reinterpret_cast<const half2*>(&u.x));
-  const float2 b = __half22float2(*reinterpret_cast<const half2*>(&u.y));
-  v[0] = a.x;
-  v[1] = a.y;
-  v[2] = b.x;
-  v[3] = b.y;
-}
-__device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  v[0] = a.x;
-  v[1] = a.y;
-  v[2] = a.z;
-  v[3] = a.w;
-}
+// Four consecutive elements of a row: raw (as loaded) and as floats.
+template <typename T>
+struct Raw4;
+template <>
+struct Raw4<half> {
+  using type = uint2;
+  __device__ static type load(const half* p) { return __ldg(reinterpret_cast<const uint2*>(p)); }
+  __device__ static type zero() { return make_uint2(0u, 0u); }
+  __device__ static void to_float(const type& u, float (&v)[4]) {
+    const float2 a = __half22float2(*reinterpret_cast<const half2*>(&u.x));
+    const float2 b = __half22float2(*reinterpret_cast<const half2*>(&u.y));
+    v[0] = a.x;
+    v[1] = a.y;
+    v[2] = b.x;
+    v[3] = b.y;
+  }
+};
+template <>
+struct Raw4<float> {
+  using type = float4;
+  __device__ static type load(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+  __device__ static type zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ static void to_float(const type& u, float (&v)[4]) {
+    v[0] = u.x;
+    v[1] = u.y;
+    v[2] = u.z;
+    v[3] = u.w;
+  }
+};
+__device__ __forceinline__ void load4(const half* p, float (&v)[4]) { Raw4<half>::to_float(Raw4<half>::load(p), v); }
+__device__ __forceinline__ void load4(const float* p, float (&v)[4]) { Raw4<float>::to_float(Raw4<float>::load(p), v); }
 
 // grid: one CTA per (batch, kv-head) row. Warp w takes batches of 8 text
 // tokens (batch w, w + 8, ...); lane l holds channels 4 l .. 4 l + 3 of the
@@ -71,16 +85,34 @@ __global__ void __launch_bounds__(kThreads) k_text_merge(const T* __restrict__ q
   }
   const T* kr = kt + (size_t)row * n_text * kD + 4 * lane;
   const T* vr = vt + (size_t)row * n_text * kD + 4 * lane;
+  using R = Raw4<T>;
+  // the next pass's keys and values are loaded while this pass computes
+  typename R::type kraw[kBatch], vraw[kBatch];
+#pragma unroll
+  for (int u = 0; u < kBatch; ++u) {
+    const int j = kBatch * warp + u;
+    kraw[u] = j < n_text ? R::load(kr + (size_t)j * kD) : R::zero();
+    vraw[u] = j < n_text ? R::load(vr + (size_t)j * kD) : R::zero();
+  }
   // every warp runs every pass (a pass past the end masks all its tokens): the
   // butterfly's shuffles must not sit in a loop whose trip count the compiler
   // sees as per-thread, where each costs several times its latency
   for (int jb = 0; jb < n_text; jb += kBatch * kWarps) {
     const int j0 = jb + kBatch * warp;
+    typename R::type kcur[kBatch], vcur[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      kcur[u] = kraw[u];
+      vcur[u] = vraw[u];
+      const int j = j0 + kBatch * kWarps + u;
+      kraw[u] = j < n_text ? R::load(kr + (size_t)j * kD) : R::zero();
+      vraw[u] = j < n_text ? R::load(vr + (size_t)j * kD) : R::zero();
+    }
     float dv[kBatch * kG];  // partial dots, index 4 token + head
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
-      float kv[4] = {0.f, 0.f, 0.f, 0.f};
-      if (j0 + u < n_text) load4(kr + (size_t)(j0 + u) * kD, kv);
+      float kv[4];
+      R::to_float(kcur[u], kv);
 #pragma unroll
       for (int h = 0; h < kG; ++h)
         dv[kG * u + h] = qv[h][0] * kv[0] + qv[h][1] * kv[1] + qv[h][2] * kv[2] + qv[h][3] * kv[3];
@@ -118,10 +150,7 @@ __global__ void __launch_bounds__(kThreads) k_text_merge(const T* __restrict__ q
     // every lane updates its 4 channels of all 4 heads
     float vv[kBatch][4];
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      vv[u][0] = vv[u][1] = vv[u][2] = vv[u][3] = 0.f;
-      if (j0 + u < n_text) load4(vr + (size_t)(j0 + u) * kD, vv[u]);
-    }
+    for (int u = 0; u < kBatch; ++u) R::to_float(vcur[u], vv[u]);
 #pragma unroll
     for (int h = 0; h < kG; ++h) {
       const float sch = __shfl_sync(0xffffffffu, sc, h);
