@@ -318,9 +318,16 @@ cq_status cq_decode_attn_mixed(const void* q, cq_dtype dt, const uint8_t* k_code
   CQ_TRY(check_ptr(workspace));
   cq::DecodeArgs a = make_args(q, k_codes, k_alpha, k_scale, v_codes, v_alpha, v_scale, B, Hq, Hkv, n_vis, d,
                                bits, softmax_scale, calib, out);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (bits == 1 && choose_1bit(n_vis, B * Hkv, false) == Kernel1::kRow) {
+    // one launch: the row kernel attends the text tokens after the quantized ones
+    a.k_text = k_text;
+    a.v_text = v_text;
+    a.n_text = n_text;
+    return cuda_status(cq::launch_decode_row(a, dt, s));
+  }
   a.part_o = static_cast<float*>(workspace);
   a.part_lse = a.part_o + (size_t)B * Hq * kD;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = bits != 1 ? cq::launch_decode_ring(a, dt, s) : launch_decode_1bit(a, dt, s);
   if (e == cudaErrorNotSupported) return CQ_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return CQ_ERR_CUDA;

@@ -54,6 +54,7 @@
 #include "kernels.h"
 #include "mma_util.cuh"
 #include "tc.cuh"
+#include "text_attend.cuh"
 
 namespace cq {
 
@@ -487,6 +488,33 @@ __global__ void __launch_bounds__(kThreads, 2)
           *reinterpret_cast<float2*>(part + (q * kG + g) * kD + 64 * hc + 8 * jn + 2 * tq) = make_float2(v[0], v[1]);
       }
     }
+
+    // ---- 8. text tokens of a mixed cache (none in a plain decode): each warp
+    // attends its share of the row's full-precision tokens with an online softmax
+    // on the raw logits sigma q.k; merged below by log-sum-exp. The ring is idle
+    // now (every chunk issued has been consumed) and holds the warps' parts.
+    float* t_acc = reinterpret_cast<float*>(ring);  // [warp][head][channel]
+    float* t_ml = t_acc + 8 * kG * kD;              // [warp][head][running maximum, sum of weights]
+    if (a.n_text > 0) {
+      float qv[kG][4];
+#pragma unroll
+      for (int hh = 0; hh < kG; ++hh)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) qv[hh][c] = DT<T>::f(sRows[hh * kD + 4 * lane + c]);
+      float tm[kG], tl[kG], tacc[kG][4];
+      const size_t toff = (size_t)row * a.n_text * kD + 4 * lane;
+      txt::warp_text_attend<T, 8>(qv, static_cast<const T*>(a.k_text) + toff, static_cast<const T*>(a.v_text) + toff,
+                                  a.n_text, a.sigma, warp, lane, tm, tl, tacc);
+#pragma unroll
+      for (int hh = 0; hh < kG; ++hh) {
+        if (lane == 0) {
+          t_ml[(warp * kG + hh) * 2] = tm[hh];
+          t_ml[(warp * kG + hh) * 2 + 1] = tl[hh];
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) t_acc[(warp * kG + hh) * kD + 4 * lane + c] = tacc[hh][c];
+      }
+    }
     __syncthreads();
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -499,7 +527,25 @@ __global__ void __launch_bounds__(kThreads, 2)
       const float alpha = DT<T>::f(sRows[6 * kD + ch]);
       const float step = *err ? __int_as_float(0x7fc00000) : DT<T>::f(sRows[7 * kD + ch]);
       const size_t bh = (size_t)b * a.Hq + (size_t)kG * hkv + hh;
-      if (a.part_o == nullptr) {
+      if (a.n_text > 0) {
+        // quantized part: weights exp(y_i - Y), Y = ref ln 2 + cst; sum l, and
+        // sum p (alpha + s c) = alpha l + s sum c p; text parts by their maxima
+        const float Y = fmaf(F.ref[hh], 0.6931471805599453f, F.cst[hh]);
+        float M = Y;
+        for (int w8 = 0; w8 < 8; ++w8)
+          if (t_ml[(w8 * kG + hh) * 2 + 1] > 0.f) M = fmaxf(M, t_ml[(w8 * kG + hh) * 2]);
+        const float fv = expf(Y - M);
+        float num = fv * fmaf(step, sum, alpha * l), den = fv * l;
+        for (int w8 = 0; w8 < 8; ++w8) {
+          const float tlw = t_ml[(w8 * kG + hh) * 2 + 1];
+          if (tlw > 0.f) {
+            const float f = expf(t_ml[(w8 * kG + hh) * 2] - M);
+            num = fmaf(f, t_acc[(w8 * kG + hh) * kD + ch], num);
+            den = fmaf(f, tlw, den);
+          }
+        }
+        static_cast<T*>(a.out)[bh * kD + ch] = DT<T>::from_float(num / den);
+      } else if (a.part_o == nullptr) {
         static_cast<T*>(a.out)[bh * kD + ch] = DT<T>::from_float(fmaf(step, sum / l, alpha));
       } else {
         a.part_o[bh * kD + ch] = fmaf(step, sum / l, alpha);

@@ -45,6 +45,12 @@ struct DecodeArgs {
   // calibrated logits y = g(x) to part_lse [B][Hq] instead of writing out.
   float* part_o = nullptr;
   float* part_lse = nullptr;
+  // Mixed caches in one launch (k_decode_row only): full-precision text tokens
+  // [B][Hkv][n_text][d] in the input dtype, attended after the quantized ones in
+  // the same softmax (their logits sigma q.k as they are, their values as stored).
+  const void* k_text = nullptr;
+  const void* v_text = nullptr;
+  int n_text = 0;
 };
 size_t decode_generic_workspace_bytes(int B, int Hq, int n);
 cudaError_t launch_decode_generic(const DecodeArgs& a, cq_dtype dt, void* workspace,

@@ -63,13 +63,15 @@ def test_mixed_without_text_equals_plain_decode(cuda_device, bits):
     assert torch.equal(plain, mixed)
 
 
-def test_mixed_through_the_row_kernel(cuda_device):
-    """Enough (sequence, kv-head) rows for the one-CTA-per-row kernel (partial
-    mode), then the text merge; and equality with the plain decode without text."""
+@pytest.mark.parametrize("n_vis,n_text", [(700, 50), (1, 1), (257, 63), (3328, 64), (1000, 65), (8192, 300)])
+def test_mixed_through_the_row_kernel(cuda_device, n_vis, n_text):
+    """Enough (sequence, kv-head) rows for the one-CTA-per-row kernel, which
+    attends the text tokens in the same launch; and equality with the plain
+    decode without text."""
     B, Hkv = 38, 4  # 152 rows: at least one per SM
-    if cq.cq_decode_kernel_name(cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V, B, 4 * Hkv, Hkv, 700, 128, 1) != "k_decode_row":
+    if cq.cq_decode_kernel_name(cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V, B, 4 * Hkv, Hkv, n_vis, 128, 1) != "k_decode_row":
         pytest.skip("this device has more SMs than rows: the row kernel is not chosen")
-    q, k, v, kt, vt = _case(B, Hkv, 700, 50, "f16", 1, seed=77)
+    q, k, v, kt, vt = _case(B, Hkv, n_vis, n_text, "f16", 1, seed=77 + n_vis + n_text)
     qd = q.to(cuda_device)
     kq = cq.cq_quantize_kv(k.to(cuda_device), 1, cq.LAYOUT_OCTET_K)
     vq = cq.cq_quantize_kv(v.to(cuda_device), 1, cq.LAYOUT_OCTET_V)
