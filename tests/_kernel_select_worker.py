@@ -1,6 +1,7 @@
 """Runs in a child process whose environment picks the octet decode kernel
 (CALIBQ_DECODE_KERNEL is read once per process); prints one JSON line with the
-per-case row-relative errors against the fp64 oracle."""
+per-case row-relative errors against the fp64 oracle, the kernel each case ran
+and the device's SM count."""
 
 import json
 import os
@@ -21,8 +22,9 @@ from _util import f64, ref_output_rounded, row_rel_err  # noqa: E402
 
 def main():
     cases = json.loads(sys.argv[1])
-    errs = []
+    errs, names = [], []
     for n, batch, calib in cases:
+        names.append(cq.cq_decode_kernel_name(cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V, batch, 8, 2, n, 128, 1))
         q, k, v = synth.make_case(batch, 4 * 2, 2, n, 128, "f16", outliers=4, seed=n)
         kq = cq.cq_quantize_kv(k.to("cuda:0"), 1, cq.LAYOUT_OCTET_K)
         vq = cq.cq_quantize_kv(v.to("cuda:0"), 1, cq.LAYOUT_OCTET_V)
@@ -30,7 +32,8 @@ def main():
         torch.cuda.synchronize()
         ref = oracle.decode_attention(f64(q), f64(k), f64(v), 1, "f16", tuple(calib))["out"]
         errs.append(row_rel_err(out.float().cpu().numpy(), ref_output_rounded(ref, torch.float16)))
-    print(json.dumps({"errs": errs}))
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    print(json.dumps({"errs": errs, "names": names, "sms": sms}))
 
 
 if __name__ == "__main__":

@@ -33,11 +33,27 @@ def _run(kernel):
     res = subprocess.run([sys.executable, os.path.join(HERE, "_kernel_select_worker.py"), json.dumps(CASES)],
                          env=env, capture_output=True, text=True, timeout=600)
     assert res.returncode == 0, res.stderr[-2000:]
-    return json.loads(res.stdout.strip().splitlines()[-1])["errs"]
+    return json.loads(res.stdout.strip().splitlines()[-1])
+
+
+def _expected(kernel, n, rows, sms):
+    """The documented choice: a forced kernel where it takes n, else the row
+    kernel for n <= 8192 when every SM gets a row, else the cluster kernel for
+    n <= 32768, else the tcgen05 kernel."""
+    if kernel == "row" and n <= 8192:
+        return "k_decode_row"
+    if kernel == "cluster" and n <= 32768:
+        return "k_decode_mma"
+    if kernel == "tcgen05":
+        return "k_decode_octet"
+    if n <= 8192 and rows >= sms:
+        return "k_decode_row"
+    return "k_decode_mma" if n <= 32768 else "k_decode_octet"
 
 
 @pytest.mark.parametrize("kernel", [None, "row", "cluster", "tcgen05"])
 def test_octet_kernels_match_oracle(cuda_device, kernel):
-    errs = _run(kernel)
-    for (n, batch, calib), e in zip(CASES, errs):
+    r = _run(kernel)
+    for (n, batch, calib), e, name in zip(CASES, r["errs"], r["names"]):
+        assert name == _expected(kernel, n, 2 * batch, r["sms"]), (kernel, n, batch, name)
         assert e <= OUT_RTOL, (kernel, n, calib, e)

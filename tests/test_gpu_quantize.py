@@ -158,3 +158,25 @@ def test_one_bit_midpoints_across_exponent_ranges(cuda_device, dtype):
         qc = cq.cq_quantize_kv(xt.to(cuda_device), 1, layout)
         torch.cuda.synchronize()
         _check_quantized(xt, qc, 1, layout)
+
+
+@pytest.mark.parametrize("layout", ["canonical", "octet_k", "octet_v"])
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
+@pytest.mark.parametrize("n", [8192, 8193, 16384, 16385])
+def test_codes_bit_exact_across_fill_limits(cuda_device, layout, bits, n):
+    """Rows on both sides of the single-read fill's limits: 512-token tiles up
+    to n = 8192, 1024-token tiles up to 16384, the two-pass statistics + pack
+    path above. Codes, alpha and step bit for bit against the oracle."""
+    x = _cache(1, 2, n, "f16", seed=n * 3 + bits)
+    qc = cq.cq_quantize_kv(x.to(cuda_device), bits, LAYOUTS[layout])
+    torch.cuda.synchronize()
+    _check_quantized(x, qc, bits, LAYOUTS[layout])
+
+
+@pytest.mark.parametrize("n", [8193, 16385])
+def test_one_bit_f32_codes_across_fill_limits(cuda_device, n):
+    x = _cache(1, 2, n, "f32", seed=n + 5)
+    for layout in (cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V):
+        qc = cq.cq_quantize_kv(x.to(cuda_device), 1, layout)
+        torch.cuda.synchronize()
+        _check_quantized(x, qc, 1, layout)
