@@ -50,6 +50,8 @@
 // One launch per decode step, no workspace; n <= 8192 tokens per row.
 #include <float.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "mma_util.cuh"
@@ -71,6 +73,7 @@ constexpr int kMaxTiles = 32;  // n <= 8192: 8 tiles per tensor-memory lane quar
 constexpr int kWMax = (1 << 21) - 1;
 constexpr int kLimbRow = 132;  // bytes per limb row (padding spreads the fragment loads over banks)
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kTextTile = 64;  // text tokens per ring chunk (f16: 64 x 256 B keys or values)
 constexpr int kMinSmem = 80 * 1024;  // > 228 KB / 3: at most two CTAs (2 x 256 columns) per SM
 
 struct RowFixed {
@@ -103,36 +106,157 @@ __device__ __forceinline__ void gather_limbs(uint32_t p0, uint32_t p1, uint32_t 
 // Octet (0..31 within a tile) of a lane's value i (0..7): 4 tq + i, then 16 + 4 tq + i - 4.
 __device__ __forceinline__ int lane_octet(int tq, int i) { return (i < 4) ? 4 * tq + i : 12 + 4 * tq + i; }
 
-// Chunk gi (0 .. 2 nchunk - 1) of the ring: the K codes of tiles 4 gi .. 4 gi + 3,
-// then (gi >= nchunk) the V codes of tiles 4 (gi - nchunk) ..; it lands in slot
-// gi % kSlots. Tiles past the row's end arrive as zeros (tensor-copy bounds fill).
-__device__ __forceinline__ void issue_chunk(RowFixed& F, uint8_t* ring, const CUtensorMap* kmap,
-                                            const CUtensorMap* vmap, int row, int nchunk, int gi) {
+// What the ring streams for one row: the K codes, the V codes (nchunk chunks
+// each), then, for a mixed cache in f16, the keys and the values of the text
+// tokens (one chunk each per 64 tokens).
+struct Ring {
+  const CUtensorMap* kmap;
+  const CUtensorMap* vmap;
+  const CUtensorMap* ktmap;
+  const CUtensorMap* vtmap;
+  int row, nchunk, nall;
+};
+
+// Chunk gi (0 .. nall - 1) lands in slot gi % kSlots: the K codes of tiles
+// 4 gi .. 4 gi + 3, then (gi >= nchunk) the V codes of tiles 4 (gi - nchunk) ..,
+// then (gi >= 2 nchunk) alternately the keys and the values of 64 text tokens
+// as two boxes of 64 channels (8 KB each). Tiles and tokens past the row's end
+// arrive as zeros (tensor-copy bounds fill).
+__device__ __forceinline__ void issue_chunk(RowFixed& F, uint8_t* ring, const Ring& R, int gi) {
   const int s = gi % kSlots;
   atomicAdd(&F.uses[s], 1u);
   tc::mbar_arrive_expect_tx(&F.full[s], kChunkBytes);
   uint8_t* dst = ring + (size_t)s * kChunkBytes;
-  if (gi < nchunk)
-    tc::tma_load_3d(dst, kmap, 0, gi * kChunkTiles * 32, row, &F.full[s]);
-  else
-    tc::tma_load_3d(dst, vmap, 0, (gi - nchunk) * kChunkTiles * 32, row, &F.full[s]);
+  if (gi < R.nchunk) {
+    tc::tma_load_3d(dst, R.kmap, 0, gi * kChunkTiles * 32, R.row, &F.full[s]);
+  } else if (gi < 2 * R.nchunk) {
+    tc::tma_load_3d(dst, R.vmap, 0, (gi - R.nchunk) * kChunkTiles * 32, R.row, &F.full[s]);
+  } else {
+    const int tt = gi - 2 * R.nchunk;
+    const CUtensorMap* m = (tt & 1) ? R.vtmap : R.ktmap;
+    tc::tma_load_3d(dst, m, 0, (tt >> 1) * kTextTile, R.row, &F.full[s]);
+    tc::tma_load_3d(dst + kChunkBytes / 2, m, 128, (tt >> 1) * kTextTile, R.row, &F.full[s]);
+  }
 }
 
 // A warp is done reading chunk gi (its share of the slot's 8 releases is
 // `share`); the warp that completes the slot's releases issues the chunk that
 // reuses it, so no thread ever waits for a slot to drain.
-__device__ __forceinline__ void release_chunk(RowFixed& F, uint8_t* ring, const CUtensorMap* kmap,
-                                              const CUtensorMap* vmap, int row, int nchunk, int gi,
-                                              uint32_t share) {
+__device__ __forceinline__ void release_chunk(RowFixed& F, uint8_t* ring, const Ring& R, int gi, uint32_t share) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) {
     const int s = gi % kSlots;
     __threadfence_block();  // this warp's reads of the slot come before the release
     const uint32_t done = atomicAdd(&F.released[s], share) + share;
-    if (done == 8u * (uint32_t)(gi / kSlots + 1) && gi + kSlots < 2 * nchunk) {
+    if (done == 8u * (uint32_t)(gi / kSlots + 1) && gi + kSlots < R.nall) {
       __threadfence_block();
       tc::fence_proxy_async();
-      issue_chunk(F, ring, kmap, vmap, row, nchunk, gi + kSlots);
+      issue_chunk(F, ring, R, gi + kSlots);
+    }
+  }
+}
+
+// Text tokens of a mixed cache on the tensor cores (f16 keys and values in
+// the ring). Warp group warp >> 2 takes every other 64-token chunk pair, warp
+// & 3 a 16-token slice of it:
+//   S = Q K^T       A = the four query heads (rows 4..15 zero), B = key rows
+//                   from the ring (ldmatrix), f32 accumulators;
+//   online softmax  on the raw logits sigma S, per head;
+//   O^T += V^T P^T  A = value rows, transposed by ldmatrix; B = P in f16,
+//                   which is S's accumulator fragment as it stands (the lane
+//                   holding S[head g][tokens 2 tq, 2 tq + 1] is the lane whose
+//                   B fragment needs exactly those).
+// The 128-byte swizzle puts 16-byte chunk c of token row r at c ^ (r & 7).
+// On return: m = running maximum of head g (lanes with g < 4; every lane of a
+// group agrees), l = this lane's part of the head's weight sum, o[x] = rows
+// 16 x + g and 16 x + g + 8 (channels) of O^T, columns (heads) 2 tq, 2 tq + 1.
+__device__ __forceinline__ void text_mma(RowFixed& F, uint8_t* ring, uint32_t ring_u, const Ring& R,
+                                         const half* q, int ntp, int n_text, float sigma, int warp, int lane,
+                                         volatile int* err, float& m, float& l, float (&o)[8][4]) {
+  const int g = lane >> 2, tq = lane & 3, grp = warp >> 2, sl = warp & 3;
+  uint32_t qa[8][4];
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const uint32_t* qw = reinterpret_cast<const uint32_t*>(q + (g & 3) * kD + 16 * s + 2 * tq);
+    qa[s][0] = g < kG ? qw[0] : 0u;  // q[g][16 s + 2 tq ..]
+    qa[s][1] = 0u;
+    qa[s][2] = g < kG ? qw[4] : 0u;  // q[g][16 s + 8 + 2 tq ..]
+    qa[s][3] = 0u;
+  }
+  m = -FLT_MAX;
+  l = 0.f;
+#pragma unroll
+  for (int x = 0; x < 8; ++x) o[x][0] = o[x][1] = o[x][2] = o[x][3] = 0.f;
+  const int mat = lane >> 3, r = lane & 7;
+  const uint32_t rowoff = (uint32_t)(16 * sl + 8 * (mat >> 1) + r) * 128u;  // this lane's ldmatrix row
+  for (int tp0 = 0; tp0 < ntp; tp0 += 2) {
+    const int tp = tp0 + grp, gk = 2 * R.nchunk + 2 * tp, gv = gk + 1;
+    const bool act = tp < ntp;
+    float sacc[2][4];
+#pragma unroll
+    for (int n = 0; n < 2; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+    if (act) {
+      warp_wait_copies(&F.full[gk % kSlots], (uint32_t)(gk / kSlots) & 1u, err);
+      const uint32_t kt = ring_u + (uint32_t)((gk % kSlots) * kChunkBytes) + rowoff;
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {  // channels 16 s .. 16 s + 15
+        const uint32_t c = (uint32_t)(2 * (s & 3) + (mat & 1));
+        uint32_t b[4];
+        ldsm_x4(kt + (uint32_t)((s >> 2) * (kChunkBytes / 2)) + ((c ^ (uint32_t)r) << 4), b);
+        mma_f16(sacc[0], qa[s], b[0], b[1]);
+        mma_f16(sacc[1], qa[s], b[2], b[3]);
+      }
+      release_chunk(F, ring, R, gk, 2);  // four warps per chunk
+    }
+    // logits of head g at tokens 64 tp + 16 sl + 8 n + 2 tq + e
+    const int t0 = kTextTile * tp + 16 * sl + 2 * tq;
+    float x[2][2], tmax = -FLT_MAX;
+    bool ok[2][2];
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        ok[n][e] = act && g < kG && t0 + 8 * n + e < n_text;
+        x[n][e] = ok[n][e] ? sigma * sacc[n][e] : -FLT_MAX;
+        tmax = fmaxf(tmax, x[n][e]);
+      }
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+    const float mnew = fmaxf(m, tmax);
+    const float sc = ex2_approx((m - mnew) * kLog2e);  // 1 while nothing was seen, 0 on the first tokens
+    uint32_t pb[2];
+    float psum = 0.f;
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+      const float p0 = ok[n][0] ? ex2_approx((x[n][0] - mnew) * kLog2e) : 0.f;
+      const float p1 = ok[n][1] ? ex2_approx((x[n][1] - mnew) * kLog2e) : 0.f;
+      const __half2 h2 = __floats2half2_rn(p0, p1);
+      pb[n] = *reinterpret_cast<const uint32_t*>(&h2);
+      const float2 back = __half22float2(h2);  // the weights the MMA uses
+      psum += back.x + back.y;
+    }
+    l = fmaf(l, sc, psum);
+    m = mnew;
+    // O^T columns are heads 2 tq, 2 tq + 1: their factors sit in lanes 8 tq, 8 tq + 4
+    const float sc0 = __shfl_sync(0xffffffffu, sc, 8 * tq), sc1 = __shfl_sync(0xffffffffu, sc, 8 * tq + 4);
+#pragma unroll
+    for (int xx = 0; xx < 8; ++xx) {
+      o[xx][0] *= sc0;
+      o[xx][1] *= sc1;
+      o[xx][2] *= sc0;
+      o[xx][3] *= sc1;
+    }
+    if (act) {
+      warp_wait_copies(&F.full[gv % kSlots], (uint32_t)(gv / kSlots) & 1u, err);
+      const uint32_t vt = ring_u + (uint32_t)((gv % kSlots) * kChunkBytes) + rowoff;
+#pragma unroll
+      for (int xx = 0; xx < 8; ++xx) {  // channels 16 xx .. 16 xx + 15
+        const uint32_t c = (uint32_t)(2 * (xx & 3) + (mat & 1));
+        uint32_t av[4];
+        ldsm_x4_trans(vt + (uint32_t)((xx >> 2) * (kChunkBytes / 2)) + ((c ^ (uint32_t)r) << 4), av);
+        mma_f16(o[xx], av, pb[0], pb[1]);
+      }
+      release_chunk(F, ring, R, gv, 2);
     }
   }
 }
@@ -143,7 +267,8 @@ __device__ __forceinline__ void release_chunk(RowFixed& F, uint8_t* ring, const 
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 2)
     k_decode_row(const __grid_constant__ DecodeArgs a, uint32_t tmem_cols, const __grid_constant__ CUtensorMap kmap,
-                 const __grid_constant__ CUtensorMap vmap) {
+                 const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap ktmap,
+                 const __grid_constant__ CUtensorMap vtmap) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* ring = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   RowFixed& F = *reinterpret_cast<RowFixed*>(ring + (size_t)kSlots * kChunkBytes);
@@ -156,6 +281,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int n = a.n;
   const int nt = (n + kTile - 1) / kTile;                   // tiles of the row
   const int nchunk = (nt + kChunkTiles - 1) / kChunkTiles;  // ring chunks per side
+  // f16 text tokens of a mixed cache stream through the ring after the V codes
+  // and meet the tensor cores; f32 ones are read directly by the warps
+  constexpr bool kTextMma = std::is_same<T, half>::value;
+  const int ntp = kTextMma ? (a.n_text + kTextTile - 1) / kTextTile : 0;  // text key / value chunk pairs
+  const Ring R{&kmap, &vmap, &ktmap, &vtmap, row, nchunk, 2 * nchunk + 2 * ntp};
   volatile int* err = &F.err;
 
   // ---- 1. barriers, tensor memory, the query and statistics rows, the first chunks
@@ -177,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc::bulk_load(F.stage + 5 * kRow, static_cast<const uint8_t*>(a.k_scale) + stat, kRow, &F.bar_rows);
     tc::bulk_load(F.stage + 6 * kRow, static_cast<const uint8_t*>(a.v_alpha) + stat, kRow, &F.bar_rows);
     tc::bulk_load(F.stage + 7 * kRow, static_cast<const uint8_t*>(a.v_scale) + stat, kRow, &F.bar_rows);
-    for (int gi = 0; gi < kSlots && gi < 2 * nchunk; ++gi) issue_chunk(F, ring, &kmap, &vmap, row, nchunk, gi);
+    for (int gi = 0; gi < kSlots && gi < R.nall; ++gi) issue_chunk(F, ring, R, gi);
   }
   if (warp == 0) {
     tc::tmem_alloc(&F.tmem_base, tmem_cols);
@@ -285,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
           for (int jn = 0; jn < 4; ++jn) bk[cc][jn][0] = bk[cc][jn][1] = 0u;
       }
-      if (act) release_chunk(F, ring, &kmap, &vmap, row, nchunk, c, 2);  // K side: four warps per chunk
+      if (act) release_chunk(F, ring, R, c, 2);  // K side: four warps per chunk
       const bool ragged = kTile * (j + 1) > n;
       const uint32_t col0 = tlane + (uint32_t)(32 * (j >> 2));
 #pragma unroll
@@ -454,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int jn = 0; jn < 8; ++jn) bv[jn][0] = bv[jn][1] = 0u;
       }
-      release_chunk(F, ring, &kmap, &vmap, row, nchunk, gi, 1);  // V side: all eight warps per chunk
+      release_chunk(F, ring, R, gi, 1);  // V side: all eight warps per chunk
       uint32_t fr[32];  // A fragments of the tile's 8 bit positions (zero past the row's end)
       tc::ld_x16(tlane + (uint32_t)(32 * c), *reinterpret_cast<uint32_t(*)[16]>(&fr[0]));
       tc::ld_x16(tlane + (uint32_t)(32 * c + 16), *reinterpret_cast<uint32_t(*)[16]>(&fr[16]));
@@ -491,28 +621,51 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     // ---- 8. text tokens of a mixed cache (none in a plain decode): each warp
     // attends its share of the row's full-precision tokens with an online softmax
-    // on the raw logits sigma q.k; merged below by log-sum-exp. The ring is idle
-    // now (every chunk issued has been consumed) and holds the warps' parts.
+    // on the raw logits sigma q.k; merged below by log-sum-exp. Once every warp
+    // is past the ring's last chunk, the ring holds the warps' parts.
     float* t_acc = reinterpret_cast<float*>(ring);  // [warp][head][channel]
     float* t_ml = t_acc + 8 * kG * kD;              // [warp][head][running maximum, sum of weights]
     if (a.n_text > 0) {
-      float qv[kG][4];
-#pragma unroll
-      for (int hh = 0; hh < kG; ++hh)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) qv[hh][c] = DT<T>::f(sRows[hh * kD + 4 * lane + c]);
-      float tm[kG], tl[kG], tacc[kG][4];
-      const size_t toff = (size_t)row * a.n_text * kD + 4 * lane;
-      txt::warp_text_attend<T, 8>(qv, static_cast<const T*>(a.k_text) + toff, static_cast<const T*>(a.v_text) + toff,
-                                  a.n_text, a.sigma, warp, lane, tm, tl, tacc);
-#pragma unroll
-      for (int hh = 0; hh < kG; ++hh) {
-        if (lane == 0) {
-          t_ml[(warp * kG + hh) * 2] = tm[hh];
-          t_ml[(warp * kG + hh) * 2 + 1] = tl[hh];
+      if constexpr (kTextMma) {
+        float tm, tl, o[8][4];
+        text_mma(F, ring, ring_u, R, sRows, ntp, a.n_text, a.sigma, warp, lane, err, tm, tl, o);
+        tl += __shfl_xor_sync(0xffffffffu, tl, 1);
+        tl += __shfl_xor_sync(0xffffffffu, tl, 2);
+        __syncthreads();  // the ring's text chunks are all read
+        if (g < kG && tq == 0) {
+          t_ml[(warp * kG + g) * 2] = tm;
+          t_ml[(warp * kG + g) * 2 + 1] = tl;
         }
+        if (tq < 2) {
+          float* h0 = t_acc + (warp * kG + 2 * tq) * kD;  // head 2 tq; head 2 tq + 1 follows
 #pragma unroll
-        for (int c = 0; c < 4; ++c) t_acc[(warp * kG + hh) * kD + 4 * lane + c] = tacc[hh][c];
+          for (int xx = 0; xx < 8; ++xx) {
+            h0[16 * xx + g] = o[xx][0];
+            h0[kD + 16 * xx + g] = o[xx][1];
+            h0[16 * xx + g + 8] = o[xx][2];
+            h0[kD + 16 * xx + g + 8] = o[xx][3];
+          }
+        }
+      } else {
+        float qv[kG][4];
+#pragma unroll
+        for (int hh = 0; hh < kG; ++hh)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) qv[hh][c] = DT<T>::f(sRows[hh * kD + 4 * lane + c]);
+        float tm[kG], tl[kG], tacc[kG][4];
+        const size_t toff = (size_t)row * a.n_text * kD + 4 * lane;
+        txt::warp_text_attend<T, 8>(qv, static_cast<const T*>(a.k_text) + toff,
+                                    static_cast<const T*>(a.v_text) + toff, a.n_text, a.sigma, warp, lane, tm, tl,
+                                    tacc);
+#pragma unroll
+        for (int hh = 0; hh < kG; ++hh) {
+          if (lane == 0) {
+            t_ml[(warp * kG + hh) * 2] = tm[hh];
+            t_ml[(warp * kG + hh) * 2 + 1] = tl[hh];
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) t_acc[(warp * kG + hh) * kD + 4 * lane + c] = tacc[hh][c];
+        }
       }
     }
     __syncthreads();
@@ -590,7 +743,14 @@ cudaError_t run_row(const DecodeArgs& a, cudaStream_t stream) {
       !encode_3d(&vmap, a.v_codes, 128, (uint64_t)nt * 32, (uint64_t)rows, kChunkTiles * 32,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  k_decode_row<T><<<rows, kThreads, smem, stream>>>(a, cols, kmap, vmap);
+  CUtensorMap ktmap = kmap, vtmap = vmap;  // stand-ins, never read, without f16 text tokens
+  if (std::is_same<T, half>::value && a.n_text > 0 &&
+      (!encode_3d_box(&ktmap, a.k_text, kD * sizeof(half), (uint64_t)a.n_text, (uint64_t)rows, 128, kTextTile,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+       !encode_3d_box(&vtmap, a.v_text, kD * sizeof(half), (uint64_t)a.n_text, (uint64_t)rows, 128, kTextTile,
+                      CU_TENSOR_MAP_SWIZZLE_128B)))
+    return cudaErrorInvalidValue;
+  k_decode_row<T><<<rows, kThreads, smem, stream>>>(a, cols, kmap, vmap, ktmap, vtmap);
   return cudaGetLastError();
 }
 

@@ -253,7 +253,12 @@ cq_status cq_decode_attn_mixed_workspace_size(int B, int Hq, int d, size_t* byte
  *   k_text, v_text: [B][Hkv][n_text][d] in `dt` (may be NULL when n_text = 0);
  *   q, out: [B][Hq][d] in `dt`; Hq = 4 * Hkv; d = 128;
  *   n_vis <= 32768; workspace: cq_decode_attn_mixed_workspace_size bytes.
- * Two launches on `stream` (visual partial, then text + merge).
+ * With 1-bit codes, when cq_decode_kernel_name names "k_decode_row", one
+ * launch on `stream`: that kernel attends the text tokens after the visual
+ * ones (f16 keys and values on the tensor cores, probabilities rounded to f16
+ * for the value product; f32 on the CUDA cores). Otherwise two launches
+ * (visual partial result into the workspace, then text + merge). The
+ * workspace is required in both cases.
  */
 cq_status cq_decode_attn_mixed(const void* q, cq_dtype dt, const uint8_t* k_codes, const void* k_alpha,
                                const void* k_scale, const uint8_t* v_codes, const void* v_alpha,

@@ -63,15 +63,25 @@ def test_mixed_without_text_equals_plain_decode(cuda_device, bits):
     assert torch.equal(plain, mixed)
 
 
-@pytest.mark.parametrize("n_vis,n_text", [(700, 50), (1, 1), (257, 63), (3328, 64), (1000, 65), (8192, 300)])
-def test_mixed_through_the_row_kernel(cuda_device, n_vis, n_text):
-    """Enough (sequence, kv-head) rows for the one-CTA-per-row kernel, which
-    attends the text tokens in the same launch; and equality with the plain
-    decode without text."""
-    B, Hkv = 38, 4  # 152 rows: at least one per SM
+ROW_CASES = [("f16", 700, 50), ("f16", 1, 1), ("f16", 257, 63), ("f16", 3328, 64), ("f16", 1000, 65),
+             ("f16", 8192, 300), ("f16", 64, 129), ("f16", 2048, 1024), ("f32", 700, 50), ("f32", 8192, 300)]
+
+
+def _row_kernel_or_skip(B, Hkv, n_vis):
     if cq.cq_decode_kernel_name(cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V, B, 4 * Hkv, Hkv, n_vis, 128, 1) != "k_decode_row":
         pytest.skip("this device has more SMs than rows: the row kernel is not chosen")
-    q, k, v, kt, vt = _case(B, Hkv, n_vis, n_text, "f16", 1, seed=77 + n_vis + n_text)
+
+
+@pytest.mark.parametrize("dtype,n_vis,n_text", ROW_CASES)
+def test_mixed_through_the_row_kernel(cuda_device, dtype, n_vis, n_text):
+    """Enough (sequence, kv-head) rows for the one-CTA-per-row kernel, which
+    attends the text tokens in the same launch (f16: through the ring and the
+    tensor cores, 64 tokens per chunk, whole and partial chunks, odd and even
+    chunk-pair counts; f32: on the CUDA cores); and equality with the plain
+    decode without text."""
+    B, Hkv = 38, 4  # 152 rows: at least one per SM
+    _row_kernel_or_skip(B, Hkv, n_vis)
+    q, k, v, kt, vt = _case(B, Hkv, n_vis, n_text, dtype, 1, seed=77 + n_vis + n_text)
     qd = q.to(cuda_device)
     kq = cq.cq_quantize_kv(k.to(cuda_device), 1, cq.LAYOUT_OCTET_K)
     vq = cq.cq_quantize_kv(v.to(cuda_device), 1, cq.LAYOUT_OCTET_V)
@@ -80,6 +90,26 @@ def test_mixed_through_the_row_kernel(cuda_device, n_vis, n_text):
     plain = cq.cq_decode_attn(qd, kq, vq, calib=calib)
     mixed0 = cq.cq_decode_attn_mixed(qd, kq, vq, None, None, calib=calib)
     torch.cuda.synchronize()
+    ref = oracle.decode_attention_mixed(f64(q), f64(k), f64(v), f64(kt), f64(vt), 1, dtype, calib)["out"]
+    rd = torch.float16 if dtype == "f16" else torch.float32
+    assert row_rel_err(out.float().cpu().numpy(), ref_output_rounded(ref, rd)) <= OUT_RTOL
+    assert torch.equal(plain, mixed0)
+
+
+@pytest.mark.parametrize("text_scale", [0.05, 4.0])
+def test_row_kernel_text_logits_far_from_visual(cuda_device, text_scale):
+    """Text keys scaled so that the text logits sit well inside (0.05) or far
+    above (4.0) the visual ones: the log-sum-exp merge has to keep whichever
+    side carries the weight."""
+    B, Hkv = 38, 4
+    _row_kernel_or_skip(B, Hkv, 1500)
+    q, k, v, kt, vt = _case(B, Hkv, 1500, 200, "f16", 1, seed=31)
+    kt = (kt.double() * text_scale).to(torch.float16)
+    qd = q.to(cuda_device)
+    kq = cq.cq_quantize_kv(k.to(cuda_device), 1, cq.LAYOUT_OCTET_K)
+    vq = cq.cq_quantize_kv(v.to(cuda_device), 1, cq.LAYOUT_OCTET_V)
+    calib = (True, 0.8, 0.9)
+    out = cq.cq_decode_attn_mixed(qd, kq, vq, kt.to(cuda_device), vt.to(cuda_device), calib=calib)
+    torch.cuda.synchronize()
     ref = oracle.decode_attention_mixed(f64(q), f64(k), f64(v), f64(kt), f64(vt), 1, "f16", calib)["out"]
     assert row_rel_err(out.float().cpu().numpy(), ref_output_rounded(ref, torch.float16)) <= OUT_RTOL
-    assert torch.equal(plain, mixed0)
