@@ -189,50 +189,63 @@ __global__ void __launch_bounds__(kThreads) k_pack_octet_k(
   k_pack_octet_k_tile<T>(x, n, row, blockIdx.y, tile_tokens, s_alpha, s_beta, s_inv, codes);
 }
 
-// OCTET_V layout (bits = 1): a warp owns 32 consecutive tokens; lane l reads
-// token l's row and the warp ballots each channel into one 32-token word,
-// which is bytes 4q..4q+3 of that channel's 32-byte row in the 256-token tile.
+// OCTET_V layout (bits = 1): channel j's 32-byte row of a 256-token layout
+// tile is the 256-bit vector of its codes in token order. The CTA takes its
+// tile 256 tokens at a time; warp w owns tokens 32 w .. 32 w + 31, i.e. word w
+// of every channel's row. Lane l reads channels 8 (l % 16) .. + 7 of tokens
+// 16 (l / 16) .. + 15 (so each load instruction covers two whole token rows),
+// sets one bit per token in a 16-bit word per channel, and the two half-warps
+// join their halves with one exchange. The 4 KB layout tile is assembled in
+// shared memory (rows padded to 9 words, which keeps both the assembly and the
+// read-out within two-to-four-way bank conflicts) and written out with
+// coalesced 4-byte stores.
 template <typename T>
 __device__ __forceinline__ void k_pack_octet_v_tile(const T* __restrict__ x, int n, int row, int tile, int tile_tokens,
     const float* s_alpha, const float* s_beta, const float* s_inv, uint8_t* __restrict__ codes) {
   __shared__ float s_hi[kD], s_lo[kD];  // alpha + beta per channel as an exact pair
+  __shared__ uint32_t stage[kD * 9];    // [channel][word 0..7, padding]
   if (threadIdx.x < kD) two_sum(s_alpha[threadIdx.x], s_beta[threadIdx.x], s_hi[threadIdx.x], s_lo[threadIdx.x]);
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, cg = lane & 15, hh = lane >> 4;
+  float hi[8], lo[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    hi[e] = s_hi[8 * cg + e];
+    lo[e] = s_lo[8 * cg + e];
+  }
   const int n_pad = (n + 255) / 256 * 256;
-  const int b0 = tile * (tile_tokens / 32), b1 = min(n_pad / 32, b0 + tile_tokens / 32);
-  const T* xr = x + (size_t)row * n * kD;
+  const int v0 = tile * (tile_tokens / 256), v1 = min(n_pad / 256, v0 + tile_tokens / 256);
+  const T* xr = x + (size_t)row * n * kD + 8 * cg;
   uint8_t* cr = codes + (size_t)row * (n_pad / 256) * 4096;
-  // Every warp runs every pass (the trip count depends on the tile only): a
-  // ballot inside a loop whose trip count the compiler sees as per-thread costs
-  // several times its latency. A pass past the tile's end ballots zeros and
-  // stores nothing.
-  const int warp_u = __shfl_sync(0xffffffffu, warp, 0);
-  for (int pass = 0; pass < b1 - b0; pass += kThreads / 32) {
-    const int blk = b0 + pass + warp_u;
-    const int i = blk * 32 + lane;
-    const bool live = blk < b1 && i < n;
-    uint32_t words[4] = {0, 0, 0, 0};  // channels lane, lane+32, lane+64, lane+96
-#pragma unroll 4
-    for (int cg = 0; cg < kD / 8; ++cg) {
-      float v[8];
-      if (live) load8(xr + (size_t)i * kD + cg * 8, v);
+  for (int vt = v0; vt < v1; ++vt) {
+    const int tok0 = vt * 256 + 32 * warp + 16 * hh;
+    uint32_t acc[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // bit i: token tok0 + i
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int j = cg * 8 + e;
-        const uint32_t code = live ? code1(v[e], s_hi[j], s_lo[j]) : 0u;
-        const uint32_t bal = __ballot_sync(0xffffffffu, code);
-        if ((j & 31) == lane) words[j >> 5] = bal;
+    for (int i = 0; i < 16; ++i) {
+      if (tok0 + i < n) {
+        float v[8];
+        load8(xr + (size_t)(tok0 + i) * kD, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] |= code1(v[e], hi[e], lo[e]) << i;
       }
     }
-    if (blk < b1) {
-      const int vt = blk >> 3, q = blk & 7;  // 256-token tile of the layout, word within its 32-byte row
+    uint32_t word[8];
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const int j = w * 32 + lane;
-        *reinterpret_cast<uint32_t*>(cr + (size_t)vt * 4096 + j * 32 + q * 4) = words[w];
-      }
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t other = __shfl_xor_sync(0xffffffffu, acc[e], 16);
+      word[e] = hh ? (other | (acc[e] << 16)) : (acc[e] | (other << 16));
     }
+    // lane (cg, hh) stores channels 8 cg + 4 hh .. 8 cg + 4 hh + 3
+#pragma unroll
+    for (int j = 0; j < 4; ++j) stage[(8 * cg + 4 * hh + j) * 9 + warp] = hh ? word[4 + j] : word[j];
+    __syncthreads();
+    uint32_t* dst = reinterpret_cast<uint32_t*>(cr + (size_t)vt * 4096);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int w = (int)threadIdx.x + kThreads * k;  // word w: channel w / 8, word w % 8 of its row
+      dst[w] = stage[(w >> 3) * 9 + (w & 7)];
+    }
+    __syncthreads();
   }
 }
 
@@ -403,18 +416,22 @@ cudaError_t launch_fill(const T* x, int rows, int n, uint8_t* codes, T* alpha, T
   const int cl = (n + tile - 1) / tile;
   // Dynamic shared memory only to cap residency at 4 CTAs per SM: 4 x 148 tiles
   // of 512 tokens x 256 B = 76 MB in flight, inside the 126 MB L2, so each
-  // tile's second read hits L2 (at 1024-token tiles the cap is the same).
-  constexpr int kPad = 12 * 1024;
-  static bool attr_set = false;  // benign race: every caller sets the same values
-  if (!attr_set) {
+  // tile's second read hits L2 (at 1024-token tiles the cap is the same). The
+  // pad brings static + dynamic to 46 KB: more than 228 KB / 5, and within the
+  // 48 KB a launch may use without opting in.
+  constexpr int kTotal = 46 * 1024;
+  static int pad = -1;  // benign race: every caller computes the same values
+  if (pad < 0) {
     cudaError_t e = cudaFuncSetAttribute(k_fill<T, BITS, LAYOUT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaFuncAttributes fa;
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, k_fill<T, BITS, LAYOUT>);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    pad = fa.sharedSizeBytes < (size_t)kTotal ? kTotal - (int)fa.sharedSizeBytes : 0;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(rows * cl), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kPad;
+  cfg.dynamicSmemBytes = (size_t)pad;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
