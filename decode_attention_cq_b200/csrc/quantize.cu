@@ -32,7 +32,7 @@ __device__ __forceinline__ void tile_minmax(const T* __restrict__ xrow, int i0, 
     mx[e] = -FLT_MAX;
   }
   const T* base = xrow + cg * 8;
-#pragma unroll 4
+#pragma unroll 8
   for (int i = i0 + r; i < i1; i += kRpi) {
     float v[8];
     load8(base + (size_t)i * kD, v);
@@ -356,7 +356,8 @@ __global__ void __launch_bounds__(kThreads) k_pack_octet_v_b(
 }
 
 // Single-read fill: one thread-block cluster per row, one CTA per tile of
-// kFillTile tokens. Each CTA takes the min / max of its tile, pushes them to
+// tile_tokens tokens. Each CTA first asks L2 for its whole tile (bulk
+// prefetches, no registers held), takes the min / max of the tile, pushes them to
 // every CTA of the cluster (distributed shared memory), folds the row's
 // statistics from what it received (the same fold as the two-launch path, so
 // alpha, step and codes are identical) and packs its own tile. The pack re-reads
@@ -374,6 +375,15 @@ __global__ void __launch_bounds__(kThreads, 4) k_fill(const T* __restrict__ x, i
   const int row = blockIdx.x / cl;
   tc::cluster_arrive_relaxed();  // matched by the wait before the first peer store
   const int i0 = (int)rank * tile_tokens, i1 = min(n, i0 + tile_tokens);
+  {
+    // the whole tile is requested into L2 at once (16 KB per request), so HBM
+    // sees every resident CTA's tile in flight; both passes below read from L2
+    constexpr int kReq = 16 * 1024;
+    const char* tile0 = reinterpret_cast<const char*>(x + ((size_t)row * n + i0) * kD);
+    const int bytes = (i1 - i0) * kD * (int)sizeof(T);
+    if ((int)threadIdx.x * kReq < bytes)
+      tc::prefetch_l2_bulk(tile0 + (size_t)threadIdx.x * kReq, (uint32_t)min(kReq, bytes - (int)threadIdx.x * kReq));
+  }
   float a, b;
   tile_minmax<T>(x + (size_t)row * n * kD, i0, i1, a, b);
   tc::cluster_wait();  // every CTA of the cluster is running

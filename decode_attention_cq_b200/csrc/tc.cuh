@@ -168,6 +168,13 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 }
 // One box of a 3-D tensor map (innermost coordinate first) into shared memory,
 // completing on `mbar`. No multicast.
+// Ask L2 to fetch [src, src + bytes) from global memory (no destination, no
+// completion to wait for). src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int c0, int c1, int c2, uint64_t* mbar) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
