@@ -496,70 +496,67 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     __syncthreads();
 
-    // ---- 5. softmax weights, as the V side's A fragments, in tensor memory. A
-    // lane's 32 logit columns of a tile become, in place, its A-fragment words of
-    // the tile's 8 bit positions (column 4 k + r = register r of bit k): P =
-    // p 2^(31-k) for its own bit of every pair, a swap with lane ^ 16 (the lane
-    // holding the same head's other limbs), byte permutes into limb rows. Warp w
-    // takes the tiles it wrote on the K side; every warp runs every pass (uniform
-    // trip count), a pass past the last chunk loads and stores nothing.
+    // ---- 5./6. softmax weights and the V side, interleaved. A lane's 32 logit
+    // columns of a tile become, in place, its A-fragment words of the tile's 8
+    // bit positions (column 4 k + r = register r of bit k): P = p 2^(31-k) for its
+    // own bit of every pair, a swap with lane ^ 16 (the lane holding the same
+    // head's other limbs), byte permutes into limb rows. Warp pair (q, q + 4)
+    // (the two warps sharing a tensor-memory lane quarter) takes tiles q, q + 4,
+    // ...; warp q + 4 hc forms bit positions 4 hc .. 4 hc + 3 of the pair's next
+    // tile while it issues the MMAs of the current one, and a 64-thread barrier
+    // per tile hands the two halves over. On the V side hc picks channels
+    // 64 hc .. 64 hc + 63: A = the tile's fragments from tensor memory, B = V codes
+    // of 8 channels masked to bit k.
     const int q = warp & 3, hc = warp >> 2;
     float lsum = 0.f;
-    {
-      const float alog2 = F.alog2[h], ref = F.ref[h];
-      const uint32_t sel = lo ? 0x6240u : 0x7351u;  // bytes (limb, limb + 2) of two words: limbs 0, 2 or 1, 3
-      for (int pass = 0; pass < nchunk; pass += 2) {
-        const int jj = pass + hc, j = kChunkTiles * jj + q;  // chunk and tile
-        const bool act = jj < nchunk;
-        const bool ragged = kTile * (j + 1) > n;  // true for a tile past the row's end: every token masked
-        const uint32_t col = tlane + (uint32_t)(32 * jj);
-        uint32_t xs[32], outw[32];
-        if (act) {
-          tc::ld_x16(col, *reinterpret_cast<uint32_t(*)[16]>(&xs[0]));
-          tc::ld_x16(col + 16, *reinterpret_cast<uint32_t(*)[16]>(&xs[16]));
-          tc::wait_ld();
-        } else {
+    const float alog2 = F.alog2[h], ref = F.ref[h];
+    const uint32_t sel = lo ? 0x6240u : 0x7351u;  // bytes (limb, limb + 2) of two words: limbs 0, 2 or 1, 3
+    // this warp's half of tile 4 c + q's fragments, one bit pair (kp = 2 hc + kp2) at a time
+    auto form_half = [&](int c) {
+      const int j = kChunkTiles * c + q;
+      const bool ragged = kTile * (j + 1) > n;  // true for a tile past the row's end: every token masked
 #pragma unroll
-          for (int i = 0; i < 32; ++i) xs[i] = 0u;
+      for (int kp2 = 0; kp2 < 2; ++kp2) {
+        const int kp = 2 * hc + kp2;
+        const uint32_t col = tlane + (uint32_t)(32 * c + 8 * kp);
+        uint32_t xs[8], outw[8];
+        tc::ld_x8(col, xs);
+        tc::wait_ld();
+        const int kown = 2 * kp + (lo ? 0 : 1);
+        const float bias = (float)(31 - kown) - ref;
+        const float unscale = __int_as_float((127 - 31 + kown) << 23);  // 2^(k - 31)
+        uint32_t pown[8], poth[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float p = ex2_approx(fmaf(__uint_as_float(xs[i]), alog2, bias));
+          const bool ok = !ragged || kTile * j + 8 * lane_octet(tq, i) + kown < n;
+          pown[i] = ok ? __float2uint_rn(p) : 0u;
+          lsum = ok ? fmaf(p, unscale, lsum) : lsum;
+          poth[i] = __shfl_xor_sync(0xffffffffu, pown[i], 16);
         }
+        // bit 2 kp: the lo lanes' weights; bit 2 kp + 1: the hi lanes'
 #pragma unroll
-        for (int kp = 0; kp < 4; ++kp) {
-          const int kown = 2 * kp + (lo ? 0 : 1);
-          const float bias = (float)(31 - kown) - ref;
-          const float unscale = __int_as_float((127 - 31 + kown) << 23);  // 2^(k - 31)
-          uint32_t pown[8], poth[8];
+        for (int kk = 0; kk < 2; ++kk) {
+          uint32_t P[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float p = ex2_approx(fmaf(__uint_as_float(xs[8 * kp + i]), alog2, bias));
-            const bool ok = act && (!ragged || kTile * j + 8 * lane_octet(tq, i) + kown < n);
-            pown[i] = ok ? __float2uint_rn(p) : 0u;
-            lsum = ok ? fmaf(p, unscale, lsum) : lsum;
-            poth[i] = __shfl_xor_sync(0xffffffffu, pown[i], 16);
-          }
-          // bit 2 kp: the lo lanes' weights; bit 2 kp + 1: the hi lanes'
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {
-            uint32_t P[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) P[i] = ((kk == 0) == lo) ? pown[i] : poth[i];
-            const int b = 4 * (2 * kp + kk);
-            gather_limbs(P[0], P[1], P[2], P[3], sel, outw[b], outw[b + 1]);
-            gather_limbs(P[4], P[5], P[6], P[7], sel, outw[b + 2], outw[b + 3]);
-          }
+          for (int i = 0; i < 8; ++i) P[i] = ((kk == 0) == lo) ? pown[i] : poth[i];
+          gather_limbs(P[0], P[1], P[2], P[3], sel, outw[4 * kk], outw[4 * kk + 1]);
+          gather_limbs(P[4], P[5], P[6], P[7], sel, outw[4 * kk + 2], outw[4 * kk + 3]);
         }
-        if (act) {
-          tc::st_x32(col, outw);
-        }
+        tc::st_x8(col, outw);  // columns 8 kp .. 8 kp + 7 = bits 2 kp, 2 kp + 1
       }
       tc::wait_st();
-    }
-    tc::fence_before_sync();
-    __syncthreads();  // the other warp of each pair reads these fragments
-    tc::fence_after_sync();
+      tc::fence_before_sync();
+      switch (q) {  // barrier 1 + q: warps q and q + 4
+        case 0: tc::bar_sync_id<1>(64); break;
+        case 1: tc::bar_sync_id<2>(64); break;
+        case 2: tc::bar_sync_id<3>(64); break;
+        default: tc::bar_sync_id<4>(64); break;
+      }
+      tc::fence_after_sync();
+    };
+    form_half(0);
 
-    // ---- 6. V side: warp pair (q, q + 4) takes tiles q, q + 4, ...; hc picks
-    // channels 64 hc .. 64 hc + 63. A = the tile's fragments from tensor memory,
-    // B = V codes of 8 channels masked to bit k.
     int acc[8][4];
 #pragma unroll
     for (int jn = 0; jn < 8; ++jn) acc[jn][0] = acc[jn][1] = acc[jn][2] = acc[jn][3] = 0;
@@ -596,6 +593,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int jn = 0; jn < 8; ++jn) mma_u8u8(acc[jn], af, bv[jn][0] & msk, bv[jn][1] & msk);
       }
+      if (c + 1 < nchunk) form_half(c + 1);
     }
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);

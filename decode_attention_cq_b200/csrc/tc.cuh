@@ -151,9 +151,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* mbar, uint32_t b
                : "memory");
 }
 
-// Named barrier `id` over the first `count` threads of the CTA (a multiple of 32).
+// Named barrier `id`, complete once `count` threads (a multiple of 32) arrive.
 __device__ __forceinline__ void bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// The same with the id as an immediate, so that the compiler reserves only the
+// barriers named in the program.
+template <int kId>
+__device__ __forceinline__ void bar_sync_id(uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"n"(kId), "r"(count) : "memory");
 }
 
 // ------------------------------------------------------- bulk copies (TMA) ----
