@@ -73,7 +73,8 @@ constexpr int kMaxTiles = 32;  // n <= 8192: 8 tiles per tensor-memory lane quar
 constexpr int kWMax = (1 << 21) - 1;
 constexpr int kLimbRow = 132;  // bytes per limb row (padding spreads the fragment loads over banks)
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kTextTile = 64;  // text tokens per ring chunk (f16: 64 x 256 B keys or values)
+constexpr int kTextTile = txt::kChunkTokens;  // text tokens per ring chunk (f16: 64 x 256 B keys or values)
+static_assert(txt::kChunkBytes == 4 * 4096, "a text chunk fills one ring slot");
 constexpr int kMinSmem = 80 * 1024;  // > 228 KB / 3: at most two CTAs (2 x 256 columns) per SM
 
 struct RowFixed {
@@ -156,110 +157,21 @@ __device__ __forceinline__ void release_chunk(RowFixed& F, uint8_t* ring, const 
   }
 }
 
-// Text tokens of a mixed cache on the tensor cores (f16 keys and values in
-// the ring). Warp group warp >> 2 takes every other 64-token chunk pair, warp
-// & 3 a 16-token slice of it:
-//   S = Q K^T       A = the four query heads (rows 4..15 zero), B = key rows
-//                   from the ring (ldmatrix), f32 accumulators;
-//   online softmax  on the raw logits sigma S, per head;
-//   O^T += V^T P^T  A = value rows, transposed by ldmatrix; B = P in f16,
-//                   which is S's accumulator fragment as it stands (the lane
-//                   holding S[head g][tokens 2 tq, 2 tq + 1] is the lane whose
-//                   B fragment needs exactly those).
-// The 128-byte swizzle puts 16-byte chunk c of token row r at c ^ (r & 7).
-// On return: m = running maximum of head g (lanes with g < 4; every lane of a
-// group agrees), l = this lane's part of the head's weight sum, o[x] = rows
-// 16 x + g and 16 x + g + 8 (channels) of O^T, columns (heads) 2 tq, 2 tq + 1.
-__device__ __forceinline__ void text_mma(RowFixed& F, uint8_t* ring, uint32_t ring_u, const Ring& R,
-                                         const half* q, int ntp, int n_text, float sigma, int warp, int lane,
-                                         volatile int* err, float& m, float& l, float (&o)[8][4]) {
-  const int g = lane >> 2, tq = lane & 3, grp = warp >> 2, sl = warp & 3;
-  uint32_t qa[8][4];
-#pragma unroll
-  for (int s = 0; s < 8; ++s) {
-    const uint32_t* qw = reinterpret_cast<const uint32_t*>(q + (g & 3) * kD + 16 * s + 2 * tq);
-    qa[s][0] = g < kG ? qw[0] : 0u;  // q[g][16 s + 2 tq ..]
-    qa[s][1] = 0u;
-    qa[s][2] = g < kG ? qw[4] : 0u;  // q[g][16 s + 8 + 2 tq ..]
-    qa[s][3] = 0u;
+// The ring's text chunks as txt::text_mma consumes them: chunk gi's slot
+// once its copy has landed, and the warp's release of it (four warps per
+// text chunk).
+struct RowTextChunks {
+  RowFixed& F;
+  uint8_t* ring;
+  uint32_t ring_u;
+  const Ring& R;
+  volatile int* err;
+  __device__ __forceinline__ uint32_t wait(int gi) {
+    warp_wait_copies(&F.full[gi % kSlots], (uint32_t)(gi / kSlots) & 1u, err);
+    return ring_u + (uint32_t)((gi % kSlots) * kChunkBytes);
   }
-  m = -FLT_MAX;
-  l = 0.f;
-#pragma unroll
-  for (int x = 0; x < 8; ++x) o[x][0] = o[x][1] = o[x][2] = o[x][3] = 0.f;
-  const int mat = lane >> 3, r = lane & 7;
-  const uint32_t rowoff = (uint32_t)(16 * sl + 8 * (mat >> 1) + r) * 128u;  // this lane's ldmatrix row
-  for (int tp0 = 0; tp0 < ntp; tp0 += 2) {
-    const int tp = tp0 + grp, gk = 2 * R.nchunk + 2 * tp, gv = gk + 1;
-    const bool act = tp < ntp;
-    float sacc[2][4];
-#pragma unroll
-    for (int n = 0; n < 2; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
-    if (act) {
-      warp_wait_copies(&F.full[gk % kSlots], (uint32_t)(gk / kSlots) & 1u, err);
-      const uint32_t kt = ring_u + (uint32_t)((gk % kSlots) * kChunkBytes) + rowoff;
-#pragma unroll
-      for (int s = 0; s < 8; ++s) {  // channels 16 s .. 16 s + 15
-        const uint32_t c = (uint32_t)(2 * (s & 3) + (mat & 1));
-        uint32_t b[4];
-        ldsm_x4(kt + (uint32_t)((s >> 2) * (kChunkBytes / 2)) + ((c ^ (uint32_t)r) << 4), b);
-        mma_f16(sacc[0], qa[s], b[0], b[1]);
-        mma_f16(sacc[1], qa[s], b[2], b[3]);
-      }
-      release_chunk(F, ring, R, gk, 2);  // four warps per chunk
-    }
-    // logits of head g at tokens 64 tp + 16 sl + 8 n + 2 tq + e
-    const int t0 = kTextTile * tp + 16 * sl + 2 * tq;
-    float x[2][2], tmax = -FLT_MAX;
-    bool ok[2][2];
-#pragma unroll
-    for (int n = 0; n < 2; ++n)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        ok[n][e] = act && g < kG && t0 + 8 * n + e < n_text;
-        x[n][e] = ok[n][e] ? sigma * sacc[n][e] : -FLT_MAX;
-        tmax = fmaxf(tmax, x[n][e]);
-      }
-    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
-    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
-    const float mnew = fmaxf(m, tmax);
-    const float sc = ex2_approx((m - mnew) * kLog2e);  // 1 while nothing was seen, 0 on the first tokens
-    uint32_t pb[2];
-    float psum = 0.f;
-#pragma unroll
-    for (int n = 0; n < 2; ++n) {
-      const float p0 = ok[n][0] ? ex2_approx((x[n][0] - mnew) * kLog2e) : 0.f;
-      const float p1 = ok[n][1] ? ex2_approx((x[n][1] - mnew) * kLog2e) : 0.f;
-      const __half2 h2 = __floats2half2_rn(p0, p1);
-      pb[n] = *reinterpret_cast<const uint32_t*>(&h2);
-      const float2 back = __half22float2(h2);  // the weights the MMA uses
-      psum += back.x + back.y;
-    }
-    l = fmaf(l, sc, psum);
-    m = mnew;
-    // O^T columns are heads 2 tq, 2 tq + 1: their factors sit in lanes 8 tq, 8 tq + 4
-    const float sc0 = __shfl_sync(0xffffffffu, sc, 8 * tq), sc1 = __shfl_sync(0xffffffffu, sc, 8 * tq + 4);
-#pragma unroll
-    for (int xx = 0; xx < 8; ++xx) {
-      o[xx][0] *= sc0;
-      o[xx][1] *= sc1;
-      o[xx][2] *= sc0;
-      o[xx][3] *= sc1;
-    }
-    if (act) {
-      warp_wait_copies(&F.full[gv % kSlots], (uint32_t)(gv / kSlots) & 1u, err);
-      const uint32_t vt = ring_u + (uint32_t)((gv % kSlots) * kChunkBytes) + rowoff;
-#pragma unroll
-      for (int xx = 0; xx < 8; ++xx) {  // channels 16 xx .. 16 xx + 15
-        const uint32_t c = (uint32_t)(2 * (xx & 3) + (mat & 1));
-        uint32_t av[4];
-        ldsm_x4_trans(vt + (uint32_t)((xx >> 2) * (kChunkBytes / 2)) + ((c ^ (uint32_t)r) << 4), av);
-        mma_f16(o[xx], av, pb[0], pb[1]);
-      }
-      release_chunk(F, ring, R, gv, 2);
-    }
-  }
-}
+  __device__ __forceinline__ void release(int gi) { release_chunk(F, ring, R, gi, 2); }
+};
 
 // kmap: K codes as [rows][octets][128 B]; vmap: V codes as [rows][tiles * 32][128 B]
 // (a 128-byte line holds 4 channels' 32 bytes of a tile). Both with the
@@ -626,7 +538,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (a.n_text > 0) {
       if constexpr (kTextMma) {
         float tm, tl, o[8][4];
-        text_mma(F, ring, ring_u, R, sRows, ntp, a.n_text, a.sigma, warp, lane, err, tm, tl, o);
+        RowTextChunks chunks{F, ring, ring_u, R, err};
+        txt::text_mma(chunks, 2 * nchunk, sRows, ntp, a.n_text, a.sigma, warp, lane, tm, tl, o);
         tl += __shfl_xor_sync(0xffffffffu, tl, 1);
         tl += __shfl_xor_sync(0xffffffffu, tl, 2);
         __syncthreads();  // the ring's text chunks are all read

@@ -1,4 +1,4 @@
-// One warp's share of a decode step's attention over full-precision text tokens
+// A warp's share of a decode step's attention over full-precision text tokens
 // (mixed caches: the quantized visual tokens are attended by the octet
 // kernels, the text tokens keep their precision). Used by the text-merge
 // kernel and by the one-CTA-per-row decode kernel. Internal header.
@@ -8,12 +8,17 @@
 #include <float.h>
 #include <stdint.h>
 
+#include "mma_util.cuh"
+
 namespace cq {
 namespace txt {
 
 constexpr int kG = 4;      // query heads per kv-head
 constexpr int kBatch = 8;  // text tokens per warp pass
 constexpr int kDim = 128;  // head dimension
+constexpr int kChunkTokens = 64;     // f16 text tokens per shared-memory chunk (keys or values)
+constexpr int kChunkBytes = 16384;   // two 128-byte-swizzled boxes of 64 channels (8 KB each)
+constexpr float kLog2e = 1.4426950408889634f;
 
 // Four consecutive elements of a row: raw (as loaded) and as floats.
 template <typename T>
@@ -144,6 +149,114 @@ __device__ __forceinline__ void warp_text_attend(const float (&qv)[kG][4], const
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[h][c] = fmaf(pu, vv[u][c], acc[h][c]);
       }
+    }
+  }
+}
+
+// f16 text tokens on the tensor cores. The keys and the values of every 64
+// tokens arrive as chunks g0 + 2 p and g0 + 2 p + 1 (p = 0 .. ntp - 1), each two
+// boxes of 64 channels x 64 tokens with the 128-byte swizzle (16-byte chunk c
+// of token row r at c ^ (r & 7)). `chunks` gives a chunk's shared-memory
+// address once it has landed (wait) and takes the warp's release of it.
+// Warp group warp >> 2 (of two) takes every other chunk pair, warp & 3 a
+// 16-token slice of it:
+//   S = Q K^T       A = the four query heads (rows 4..15 zero), B = key rows
+//                   (ldmatrix), f32 accumulators;
+//   online softmax  on the raw logits sigma S, per head;
+//   O^T += V^T P^T  A = value rows, transposed by ldmatrix; B = P in f16,
+//                   which is S's accumulator fragment as it stands (the lane
+//                   holding S[head g][tokens 2 tq, 2 tq + 1] is the lane whose
+//                   B fragment needs exactly those); the weight sums use the
+//                   same rounded values.
+// On return: m = running maximum of head g (lanes with g < 4; every lane of a
+// group agrees), l = this lane's part of the head's weight sum, o[x] = rows
+// 16 x + g and 16 x + g + 8 (channels) of O^T, columns (heads) 2 tq, 2 tq + 1.
+template <class Chunks>
+__device__ __forceinline__ void text_mma(Chunks& chunks, int g0, const half* q, int ntp, int n_text, float sigma,
+                                         int warp, int lane, float& m, float& l, float (&o)[8][4]) {
+  using namespace mu;
+  const int g = lane >> 2, tq = lane & 3, grp = warp >> 2, sl = warp & 3;
+  uint32_t qa[8][4];
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const uint32_t* qw = reinterpret_cast<const uint32_t*>(q + (g & 3) * kDim + 16 * s + 2 * tq);
+    qa[s][0] = g < kG ? qw[0] : 0u;  // q[g][16 s + 2 tq ..]
+    qa[s][1] = 0u;
+    qa[s][2] = g < kG ? qw[4] : 0u;  // q[g][16 s + 8 + 2 tq ..]
+    qa[s][3] = 0u;
+  }
+  m = -FLT_MAX;
+  l = 0.f;
+#pragma unroll
+  for (int x = 0; x < 8; ++x) o[x][0] = o[x][1] = o[x][2] = o[x][3] = 0.f;
+  const int mat = lane >> 3, r = lane & 7;
+  const uint32_t rowoff = (uint32_t)(16 * sl + 8 * (mat >> 1) + r) * 128u;  // this lane's ldmatrix row
+  for (int tp0 = 0; tp0 < ntp; tp0 += 2) {
+    const int tp = tp0 + grp, gk = g0 + 2 * tp, gv = gk + 1;
+    const bool act = tp < ntp;
+    float sacc[2][4];
+#pragma unroll
+    for (int n = 0; n < 2; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+    if (act) {
+      const uint32_t kt = chunks.wait(gk) + rowoff;
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {  // channels 16 s .. 16 s + 15
+        const uint32_t c = (uint32_t)(2 * (s & 3) + (mat & 1));
+        uint32_t b[4];
+        ldsm_x4(kt + (uint32_t)((s >> 2) * (kChunkBytes / 2)) + ((c ^ (uint32_t)r) << 4), b);
+        mma_f16(sacc[0], qa[s], b[0], b[1]);
+        mma_f16(sacc[1], qa[s], b[2], b[3]);
+      }
+      chunks.release(gk);
+    }
+    // logits of head g at tokens 64 tp + 16 sl + 8 n + 2 tq + e
+    const int t0 = kChunkTokens * tp + 16 * sl + 2 * tq;
+    float x[2][2], tmax = -FLT_MAX;
+    bool ok[2][2];
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        ok[n][e] = act && g < kG && t0 + 8 * n + e < n_text;
+        x[n][e] = ok[n][e] ? sigma * sacc[n][e] : -FLT_MAX;
+        tmax = fmaxf(tmax, x[n][e]);
+      }
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+    const float mnew = fmaxf(m, tmax);
+    const float sc = ex2_approx((m - mnew) * kLog2e);  // 1 while nothing was seen, 0 on the first tokens
+    uint32_t pb[2];
+    float psum = 0.f;
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+      const float p0 = ok[n][0] ? ex2_approx((x[n][0] - mnew) * kLog2e) : 0.f;
+      const float p1 = ok[n][1] ? ex2_approx((x[n][1] - mnew) * kLog2e) : 0.f;
+      const __half2 h2 = __floats2half2_rn(p0, p1);
+      pb[n] = *reinterpret_cast<const uint32_t*>(&h2);
+      const float2 back = __half22float2(h2);  // the weights the MMA uses
+      psum += back.x + back.y;
+    }
+    l = fmaf(l, sc, psum);
+    m = mnew;
+    // O^T columns are heads 2 tq, 2 tq + 1: their factors sit in lanes 8 tq, 8 tq + 4
+    const float sc0 = __shfl_sync(0xffffffffu, sc, 8 * tq), sc1 = __shfl_sync(0xffffffffu, sc, 8 * tq + 4);
+#pragma unroll
+    for (int xx = 0; xx < 8; ++xx) {
+      o[xx][0] *= sc0;
+      o[xx][1] *= sc1;
+      o[xx][2] *= sc0;
+      o[xx][3] *= sc1;
+    }
+    if (act) {
+      const uint32_t vt = chunks.wait(gv) + rowoff;
+#pragma unroll
+      for (int xx = 0; xx < 8; ++xx) {  // channels 16 xx .. 16 xx + 15
+        const uint32_t c = (uint32_t)(2 * (xx & 3) + (mat & 1));
+        uint32_t av[4];
+        ldsm_x4_trans(vt + (uint32_t)((xx >> 2) * (kChunkBytes / 2)) + ((c ^ (uint32_t)r) << 4), av);
+        mma_f16(o[xx], av, pb[0], pb[1]);
+      }
+      chunks.release(gv);
     }
   }
 }
