@@ -336,7 +336,7 @@ def run_ours(args, world, rank, local):
                      "traffic": None if trec is None else trec["dram_bytes_per_launch"],
                      "algorithmic_bytes_per_launch": alg,
                      "kernel": kernel + ((" (text tokens in the same launch)" if kernel == "k_decode_row"
-                                          else " (partial) + k_text_merge") if n_text else "")},
+                                          else " (partial) + k_text_merge_mma") if n_text else "")},
         "cache_fill": {"ms": fill_mean, "algorithmic_bytes": fill_alg,
                        "achieved_gbs": fill_alg / (fill_mean * 1e-3) / 1e9,
                        "frac": fill_alg / (fill_mean * 1e-3) / 1e9 / peak},
