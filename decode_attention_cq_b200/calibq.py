@@ -11,6 +11,7 @@ fails loudly -- there is no CPU fallback.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 from dataclasses import dataclass
 
@@ -106,9 +107,23 @@ def _ptr(t) -> int | None:
     return None if t is None else t.data_ptr()
 
 
-def _stream(stream) -> int:
-    s = torch.cuda.current_stream() if stream is None else stream
-    return s.cuda_stream
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(stream, t: torch.Tensor | None = None) -> int:
+    """The stream handle to launch on: `stream`, else the current stream of
+    t's device (of the current device without t)."""
+    if stream is not None:
+        return stream.cuda_stream
+    if _raw_stream is not None and t is not None and t.is_cuda:
+        return _raw_stream(t.get_device())
+    return torch.cuda.current_stream().cuda_stream
+
+
+@functools.lru_cache(maxsize=64)
+def _calib(enabled: bool, tau_lo: float, tau_hi: float) -> "cq_calib":
+    # passed by value: one instance per distinct setting can be shared
+    return cq_calib(int(enabled), tau_lo, tau_hi)
 
 
 @dataclass
@@ -162,7 +177,7 @@ def cq_quantize_kv(x: torch.Tensor, bits: int, layout: int = LAYOUT_CANONICAL, *
         workspace = torch.empty(max(ws, 1), dtype=torch.uint8, device=x.device)
     _check(load().cq_quantize_kv(_ptr(x), _dt(x), B, H, n, d, bits, layout, _ptr(out.codes),
                                  _ptr(out.alpha), _ptr(out.scale), _ptr(workspace),
-                                 workspace.numel(), _stream(stream)), "cq_quantize_kv")
+                                 workspace.numel(), _stream(stream, x)), "cq_quantize_kv")
     return out
 
 
@@ -179,7 +194,7 @@ def cq_quantize_kv_noalloc(x: torch.Tensor, bits: int, layout: int = LAYOUT_CANO
             scale=torch.empty(B, H, d, dtype=x.dtype, device=x.device),
             layout=layout, bits=bits, n=n)
     _check(load().cq_quantize_kv_noalloc(_ptr(x), _dt(x), B, H, n, d, bits, layout, _ptr(out.codes),
-                                         _ptr(out.alpha), _ptr(out.scale), _stream(stream)),
+                                         _ptr(out.alpha), _ptr(out.scale), _stream(stream, x)),
            "cq_quantize_kv_noalloc")
     return out
 
@@ -211,12 +226,12 @@ def cq_decode_attn(q: torch.Tensor, k: QuantizedCache, v: QuantizedCache, *,
     if workspace is None:
         ws = cq_decode_attn_workspace_size(k.layout, v.layout, B, Hq, Hkv, n, d, k.bits)
         workspace = torch.empty(ws, dtype=torch.uint8, device=q.device) if ws else None
-    cal = cq_calib(int(bool(calib[0])), float(calib[1]), float(calib[2]))
+    cal = _calib(bool(calib[0]), float(calib[1]), float(calib[2]))
     _check(load().cq_decode_attn(_ptr(q), _dt(q), _ptr(k.codes), _ptr(k.alpha), _ptr(k.scale),
                                  k.layout, _ptr(v.codes), _ptr(v.alpha), _ptr(v.scale), v.layout,
                                  B, Hq, Hkv, n, d, k.bits, float(softmax_scale), cal, _ptr(out),
                                  _ptr(workspace), 0 if workspace is None else workspace.numel(),
-                                 _stream(stream)), "cq_decode_attn")
+                                 _stream(stream, q)), "cq_decode_attn")
     return out
 
 
@@ -242,12 +257,12 @@ def cq_decode_attn_mixed(q: torch.Tensor, k: QuantizedCache, v: QuantizedCache,
     if workspace is None:
         workspace = torch.empty(cq_decode_attn_mixed_workspace_size(B, Hq, d), dtype=torch.uint8,
                                 device=q.device)
-    cal = cq_calib(int(bool(calib[0])), float(calib[1]), float(calib[2]))
+    cal = _calib(bool(calib[0]), float(calib[1]), float(calib[2]))
     _check(load().cq_decode_attn_mixed(_ptr(q), _dt(q), _ptr(k.codes), _ptr(k.alpha), _ptr(k.scale),
                                        _ptr(v.codes), _ptr(v.alpha), _ptr(v.scale), n, k.bits,
                                        _ptr(k_text), _ptr(v_text), n_text, B, Hq, Hkv, d,
                                        float(softmax_scale), cal, _ptr(out), _ptr(workspace),
-                                       workspace.numel(), _stream(stream)), "cq_decode_attn_mixed")
+                                       workspace.numel(), _stream(stream, q)), "cq_decode_attn_mixed")
     return out
 
 
@@ -258,5 +273,5 @@ def cq_dequant(cache: QuantizedCache, *, out: torch.Tensor | None = None, stream
         out = torch.empty(B, H, n, d, dtype=cache.alpha.dtype, device=cache.alpha.device)
     _check(load().cq_dequant(_ptr(cache.codes), _ptr(cache.alpha), _ptr(cache.scale),
                              _dt(cache.alpha), cache.layout, B, H, n, d, cache.bits, _ptr(out),
-                             _stream(stream)), "cq_dequant")
+                             _stream(stream, cache.codes)), "cq_dequant")
     return out

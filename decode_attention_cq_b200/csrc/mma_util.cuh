@@ -128,8 +128,8 @@ inline EncodeTiled encode_fn() {
 }
 
 // 3-D uint8 map {inner bytes, mid, outer} with box {box_inner, box_mid, 1}.
-inline bool encode_3d_box(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
-                          uint32_t box_inner, uint32_t box_mid, CUtensorMapSwizzle swz) {
+inline bool encode_3d_box_uncached(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                                   uint32_t box_inner, uint32_t box_mid, CUtensorMapSwizzle swz) {
   const EncodeTiled fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[3] = {inner, mid, outer};
@@ -141,18 +141,47 @@ inline bool encode_3d_box(CUtensorMap* m, const void* base, uint64_t inner, uint
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same through a small per-thread cache of recent encodings: a decode loop
+// passes the same buffers every step, and an encoding depends on its arguments
+// only, so a hit returns exactly the map the encoder would write.
+inline bool encode_3d_box(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                          uint32_t box_inner, uint32_t box_mid, CUtensorMapSwizzle swz) {
+  struct Entry {
+    CUtensorMap map;
+    const void* base;
+    uint64_t inner, mid, outer;
+    uint32_t box_inner, box_mid;
+    int swz;
+    bool used;
+  };
+  constexpr int kEntries = 8;
+  thread_local Entry cache[kEntries] = {};
+  thread_local int next = 0;
+  for (Entry& e : cache)
+    if (e.used && e.base == base && e.inner == inner && e.mid == mid && e.outer == outer &&
+        e.box_inner == box_inner && e.box_mid == box_mid && e.swz == (int)swz) {
+      *m = e.map;
+      return true;
+    }
+  if (!encode_3d_box_uncached(m, base, inner, mid, outer, box_inner, box_mid, swz)) return false;
+  Entry& e = cache[next];
+  next = (next + 1) % kEntries;
+  e.map = *m;
+  e.base = base;
+  e.inner = inner;
+  e.mid = mid;
+  e.outer = outer;
+  e.box_inner = box_inner;
+  e.box_mid = box_mid;
+  e.swz = (int)swz;
+  e.used = true;
+  return true;
+}
+
 // 3-D uint8 map {inner bytes, mid, outer} with box {inner, box_mid, 1}.
 inline bool encode_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer, uint32_t box_mid,
-               CUtensorMapSwizzle swz) {
-  const EncodeTiled fn = encode_fn();
-  if (fn == nullptr) return false;
-  const cuuint64_t dims[3] = {inner, mid, outer};
-  const cuuint64_t strides[2] = {inner, inner * mid};
-  const cuuint32_t box[3] = {(cuuint32_t)inner, box_mid, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+                      CUtensorMapSwizzle swz) {
+  return encode_3d_box(m, base, inner, mid, outer, (uint32_t)inner, box_mid, swz);
 }
 
 }  // namespace mu
