@@ -12,6 +12,11 @@ from .calibq import (  # noqa: F401
     LAYOUT_CANONICAL,
     LAYOUT_OCTET_K,
     LAYOUT_OCTET_V,
+    KERNEL_AUTO,
+    KERNEL_CLUSTER,
+    KERNEL_ENV,
+    KERNEL_ROW,
+    KERNEL_TCGEN05,
     CalibqError,
     QuantizedCache,
     cq_codes_bytes,
@@ -20,6 +25,7 @@ from .calibq import (  # noqa: F401
     cq_decode_attn_mixed_workspace_size,
     cq_decode_attn_workspace_size,
     cq_decode_kernel_name,
+    cq_set_decode_kernel,
     cq_dequant,
     cq_quantize_kv,
     cq_quantize_kv_workspace_size,

@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libc
 CQ_OK, CQ_ERR_INVALID_ARG, CQ_ERR_UNSUPPORTED, CQ_ERR_WORKSPACE, CQ_ERR_CUDA = range(5)
 CQ_F16, CQ_F32 = 0, 1
 LAYOUT_CANONICAL, LAYOUT_OCTET_K, LAYOUT_OCTET_V = 0, 1, 2
+KERNEL_ENV, KERNEL_AUTO, KERNEL_ROW, KERNEL_CLUSTER, KERNEL_TCGEN05 = -1, 0, 1, 2, 3
 
 ENTRY_POINTS = (
     "cq_version",
@@ -32,6 +33,7 @@ ENTRY_POINTS = (
     "cq_quantize_kv_noalloc",
     "cq_decode_attn_workspace_size",
     "cq_decode_kernel_name",
+    "cq_set_decode_kernel",
     "cq_decode_attn",
     "cq_decode_attn_mixed_workspace_size",
     "cq_decode_attn_mixed",
@@ -59,6 +61,7 @@ _SIGS = {
     "cq_quantize_kv_noalloc": ([_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P], _I),
     "cq_decode_attn_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "cq_decode_kernel_name": ([_I, _I, _I, _I, _I, _I, _I, _I], ctypes.c_char_p),
+    "cq_set_decode_kernel": ([_I], _I),
     "cq_decode_attn": ([_P, _I, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F,
                         cq_calib, _P, _P, _SZ, _P], _I),
     "cq_decode_attn_mixed_workspace_size": ([_I, _I, _I, ctypes.POINTER(_SZ)], _I),
@@ -212,6 +215,13 @@ def cq_decode_kernel_name(k_layout: int, v_layout: int, B: int, Hq: int, Hkv: in
     """Name of the kernel cq_decode_attn launches for these arguments, or None."""
     name = load().cq_decode_kernel_name(k_layout, v_layout, B, Hq, Hkv, n, d, bits)
     return None if name is None else name.decode()
+
+
+def cq_set_decode_kernel(which: int) -> None:
+    """Force a 1-bit octet decode kernel for the rest of the process
+    (KERNEL_ROW / KERNEL_CLUSTER / KERNEL_TCGEN05), let the estimate decide
+    (KERNEL_AUTO), or go back to the environment (KERNEL_ENV)."""
+    _check(load().cq_set_decode_kernel(int(which)), "cq_set_decode_kernel")
 
 
 def cq_decode_attn(q: torch.Tensor, k: QuantizedCache, v: QuantizedCache, *,

@@ -1,4 +1,5 @@
 // The libcalibq C ABI: host-side validation and dispatch (see include/calibq.h).
+#include <atomic>
 #include <math.h>
 #include <stdlib.h>
 #include <string.h>
@@ -41,13 +42,14 @@ cq_status check_ptr(const void* p) {
 
 // 1-bit octet-layout decode kernels: "row" (one CTA per row, logits in tensor
 // memory, n <= 8192), "cluster" (a cluster of CTAs per row, n <= 32768) and
-// "tcgen05" (5th-generation tensor cores, n <= 65536). CALIBQ_DECODE_KERNEL
-// names one to use wherever it supports n; otherwise the choice is the row
-// kernel when it supports n and the batch gives every SM a row, else the
-// cluster kernel, else the tcgen05 one.
+// "tcgen05" (5th-generation tensor cores, n <= 65536). cq_set_decode_kernel,
+// else the environment variable CALIBQ_DECODE_KERNEL, may name one to use
+// wherever it supports n; otherwise the choice between the row and the cluster
+// kernel is the one with the smaller estimated step time, and the tcgen05
+// kernel takes what neither supports.
 enum class Kernel1 { kAuto, kRow, kCluster, kTcgen05 };
 
-Kernel1 forced_kernel() {
+Kernel1 env_kernel() {
   static const Kernel1 forced = [] {
     const char* v = getenv("CALIBQ_DECODE_KERNEL");
     if (v == nullptr) return Kernel1::kAuto;
@@ -57,6 +59,13 @@ Kernel1 forced_kernel() {
     return Kernel1::kAuto;
   }();
   return forced;
+}
+
+std::atomic<int> g_set_kernel{-1};  // cq_set_decode_kernel's choice; -1: none made
+
+Kernel1 forced_kernel() {
+  const int v = g_set_kernel.load(std::memory_order_relaxed);
+  return v < 0 ? env_kernel() : static_cast<Kernel1>(v);
 }
 
 int sm_count() {
@@ -70,12 +79,29 @@ int sm_count() {
   return count;
 }
 
+// Step-time estimates (microseconds on B200) of the two kernels for `rows`
+// (batch, kv-head) rows of n tokens, fitted to measurements at n = 3328 and
+// 8192 over 128 to 512 rows (every point within about 3 us). The row kernel
+// runs two CTAs per SM: t1 is a row alone on its SM, t2 a wave of two per SM,
+// and a partial last wave costs 0.6 t1 when it leaves at most one row per SM,
+// else 0.8 t2. The cluster kernel's time grows about linearly in the rows.
+double est_row_us(int n, long long rows, int sms) {
+  const double t1 = 12.8 + 0.00243 * n, t2 = 16.7 + 0.0037 * n;
+  if (rows <= sms) return t1;
+  const long long slots = 2LL * sms, full = rows / slots, rest = rows % slots;
+  if (full == 0) return t2;
+  return (double)full * t2 + (rest == 0 ? 0.0 : rest <= sms ? 0.6 * t1 : 0.8 * t2);
+}
+double est_cluster_us(int n, long long rows) { return 11.7 + (double)rows * (0.0065 + 1.77e-5 * n); }
+
 Kernel1 choose_1bit(int n, int rows, bool partial) {
   const Kernel1 f = forced_kernel();
   if (f == Kernel1::kRow && cq::decode_row_supports(n)) return Kernel1::kRow;
   if (f == Kernel1::kCluster && cq::decode_mma_supports(n)) return Kernel1::kCluster;
   if (f == Kernel1::kTcgen05 && !partial) return Kernel1::kTcgen05;
-  if (cq::decode_row_supports(n) && rows >= sm_count()) return Kernel1::kRow;
+  const int sms = sm_count();
+  if (cq::decode_row_supports(n) && sms > 0 && est_row_us(n, rows, sms) < est_cluster_us(n, rows))
+    return Kernel1::kRow;
   if (cq::decode_mma_supports(n)) return Kernel1::kCluster;
   return partial ? Kernel1::kAuto : Kernel1::kTcgen05;  // kAuto: none
 }
@@ -245,6 +271,17 @@ const char* cq_decode_kernel_name(cq_layout k_layout, cq_layout v_layout, int B,
     case Kernel1::kRow: return "k_decode_row";
     case Kernel1::kCluster: return "k_decode_mma";
     default: return "k_decode_octet";
+  }
+}
+
+cq_status cq_set_decode_kernel(cq_decode_kernel which) {
+  switch (which) {
+    case CQ_KERNEL_AUTO: g_set_kernel.store((int)Kernel1::kAuto); return CQ_OK;
+    case CQ_KERNEL_ROW: g_set_kernel.store((int)Kernel1::kRow); return CQ_OK;
+    case CQ_KERNEL_CLUSTER: g_set_kernel.store((int)Kernel1::kCluster); return CQ_OK;
+    case CQ_KERNEL_TCGEN05: g_set_kernel.store((int)Kernel1::kTcgen05); return CQ_OK;
+    case CQ_KERNEL_ENV: g_set_kernel.store(-1); return CQ_OK;
+    default: return CQ_ERR_INVALID_ARG;
   }
 }
 

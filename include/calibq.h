@@ -215,17 +215,42 @@ cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, con
  * on the current device, or NULL when the call would not launch one (invalid
  * or unsupported arguments). Host-only; reads the device's SM count once.
  *   1 bit, octet layouts: "k_decode_row" (one CTA per (sequence, kv-head) row,
- *     n <= 8192, chosen when B * Hkv >= the SM count), "k_decode_mma" (a
- *     cluster of CTAs per row, n <= 32768) or "k_decode_octet" (tcgen05,
- *     n <= 65536). The environment variable CALIBQ_DECODE_KERNEL = row |
- *     cluster | tcgen05, read once per process, forces one of them wherever it
- *     supports n.
+ *     two per SM, n <= 8192), "k_decode_mma" (a cluster of CTAs per row,
+ *     n <= 32768) or "k_decode_octet" (tcgen05, n <= 65536). Between the
+ *     first two the library takes the one with the smaller estimated step
+ *     time for B * Hkv rows of n tokens (an estimate fitted to measurements on
+ *     B200: the row kernel for long rows and full waves of two rows per SM,
+ *     the cluster kernel for short rows and for batches that leave the row
+ *     kernel a thin last wave); the tcgen05 kernel takes longer rows.
+ *     cq_set_decode_kernel, else the environment variable
+ *     CALIBQ_DECODE_KERNEL = row | cluster | tcgen05 (read once per process),
+ *     forces one of them wherever it supports n.
  *   2, 4, 8 bits, octet layouts: "k_decode_ring".
  *   Canonical layouts: "k_scores + k_softmax_v + k_merge" (three launches).
  * The returned string is static; the caller does not free it.
  */
 const char* cq_decode_kernel_name(cq_layout k_layout, cq_layout v_layout, int B, int Hq, int Hkv, int n, int d,
                                   int bits);
+
+/* 1-bit octet-layout decode kernels, for cq_set_decode_kernel. */
+typedef enum cq_decode_kernel {
+  CQ_KERNEL_ENV = -1,     /* CALIBQ_DECODE_KERNEL decides, else the estimate (the initial state) */
+  CQ_KERNEL_AUTO = 0,     /* the estimate decides, whatever the environment says */
+  CQ_KERNEL_ROW = 1,      /* "k_decode_row" wherever n <= 8192 */
+  CQ_KERNEL_CLUSTER = 2,  /* "k_decode_mma" wherever n <= 32768 */
+  CQ_KERNEL_TCGEN05 = 3   /* "k_decode_octet" (plain decodes; mixed calls choose as with AUTO) */
+} cq_decode_kernel;
+
+/*
+ * Force (or stop forcing) the 1-bit octet-layout decode kernel for every later
+ * cq_decode_attn, cq_decode_attn_mixed and cq_decode_kernel_name call of the
+ * process. A forced kernel that does not support a call's n falls back to the
+ * estimate. The kernels' outputs agree within the output tolerance, not bit
+ * for bit. Host-only; takes effect for calls made after it returns (a call
+ * racing with it on another thread may use either choice).
+ * Returns CQ_ERR_INVALID_ARG for a value outside cq_decode_kernel.
+ */
+cq_status cq_set_decode_kernel(cq_decode_kernel which);
 
 /*
  * Workspace of cq_decode_attn_mixed: the visual part's partial result

@@ -1,7 +1,7 @@
 """Runs in a child process whose environment picks the octet decode kernel
 (CALIBQ_DECODE_KERNEL is read once per process); prints one JSON line with the
-per-case row-relative errors against the fp64 oracle, the kernel each case ran
-and the device's SM count."""
+per-case row-relative errors against the fp64 oracle and the kernel each case
+ran."""
 
 import json
 import os
@@ -32,8 +32,7 @@ def main():
         torch.cuda.synchronize()
         ref = oracle.decode_attention(f64(q), f64(k), f64(v), 1, "f16", tuple(calib))["out"]
         errs.append(row_rel_err(out.float().cpu().numpy(), ref_output_rounded(ref, torch.float16)))
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    print(json.dumps({"errs": errs, "names": names, "sms": sms}))
+    print(json.dumps({"errs": errs, "names": names}))
 
 
 if __name__ == "__main__":

@@ -25,3 +25,14 @@ def cuda_device():
     if not gpu_available():
         pytest.skip("no CUDA device")
     return "cuda:0"
+
+
+@pytest.fixture
+def row_kernel(cuda_device):
+    """Force the one-CTA-per-row 1-bit decode kernel for one test (it takes
+    n <= 8192), then hand the choice back to the environment / estimate."""
+    from decode_attention_cq_b200 import calibq as cq
+
+    cq.cq_set_decode_kernel(cq.KERNEL_ROW)
+    yield cuda_device
+    cq.cq_set_decode_kernel(cq.KERNEL_ENV)

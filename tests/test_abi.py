@@ -95,6 +95,24 @@ def test_decode_kernel_name_follows_the_documented_choice(lib):
     assert cq.cq_decode_kernel_name(K, V, 1, 8, 2, 65537, 128, 1) is None
 
 
+def test_set_decode_kernel_forces_and_releases(lib):
+    K, V = cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V
+    assert lib.cq_set_decode_kernel(7) == cq.CQ_ERR_INVALID_ARG
+    try:
+        cq.cq_set_decode_kernel(cq.KERNEL_ROW)
+        assert cq.cq_decode_kernel_name(K, V, 1, 8, 2, 1000, 128, 1) == "k_decode_row"
+        assert cq.cq_decode_kernel_name(K, V, 1, 8, 2, 8193, 128, 1) == "k_decode_mma"  # row takes n <= 8192
+        cq.cq_set_decode_kernel(cq.KERNEL_CLUSTER)
+        assert cq.cq_decode_kernel_name(K, V, 64, 32, 8, 8192, 128, 1) == "k_decode_mma"
+        assert cq.cq_decode_kernel_name(K, V, 1, 8, 2, 32769, 128, 1) == "k_decode_octet"
+        cq.cq_set_decode_kernel(cq.KERNEL_TCGEN05)
+        assert cq.cq_decode_kernel_name(K, V, 64, 32, 8, 1000, 128, 1) == "k_decode_octet"
+        cq.cq_set_decode_kernel(cq.KERNEL_AUTO)
+        assert cq.cq_decode_kernel_name(K, V, 1, 8, 2, 32768, 128, 1) == "k_decode_mma"
+    finally:
+        cq.cq_set_decode_kernel(cq.KERNEL_ENV)
+
+
 def test_null_pointers_rejected_before_any_cuda_call(lib):
     st = lib.cq_quantize_kv(None, 0, 1, 1, 16, 128, 1, 0, None, None, None, None, 0, None)
     assert st == cq.CQ_ERR_INVALID_ARG

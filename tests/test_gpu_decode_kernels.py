@@ -36,24 +36,24 @@ def _run(kernel):
     return json.loads(res.stdout.strip().splitlines()[-1])
 
 
-def _expected(kernel, n, rows, sms):
-    """The documented choice: a forced kernel where it takes n, else the row
-    kernel for n <= 8192 when every SM gets a row, else the cluster kernel for
-    n <= 32768, else the tcgen05 kernel."""
+def _expected(kernel, n):
+    """The documented choice: a forced kernel where it takes n; otherwise, for
+    n <= 8192, the row or the cluster kernel (an estimate of their step times
+    decides), then the cluster kernel up to n = 32768, then the tcgen05 one."""
     if kernel == "row" and n <= 8192:
-        return "k_decode_row"
+        return {"k_decode_row"}
     if kernel == "cluster" and n <= 32768:
-        return "k_decode_mma"
+        return {"k_decode_mma"}
     if kernel == "tcgen05":
-        return "k_decode_octet"
-    if n <= 8192 and rows >= sms:
-        return "k_decode_row"
-    return "k_decode_mma" if n <= 32768 else "k_decode_octet"
+        return {"k_decode_octet"}
+    if n <= 8192:
+        return {"k_decode_row", "k_decode_mma"}
+    return {"k_decode_mma"} if n <= 32768 else {"k_decode_octet"}
 
 
 @pytest.mark.parametrize("kernel", [None, "row", "cluster", "tcgen05"])
 def test_octet_kernels_match_oracle(cuda_device, kernel):
     r = _run(kernel)
     for (n, batch, calib), e, name in zip(CASES, r["errs"], r["names"]):
-        assert name == _expected(kernel, n, 2 * batch, r["sms"]), (kernel, n, batch, name)
+        assert name in _expected(kernel, n), (kernel, n, batch, name)
         assert e <= OUT_RTOL, (kernel, n, calib, e)

@@ -67,20 +67,20 @@ ROW_CASES = [("f16", 700, 50), ("f16", 1, 1), ("f16", 257, 63), ("f16", 3328, 64
              ("f16", 8192, 300), ("f16", 64, 129), ("f16", 2048, 1024), ("f32", 700, 50), ("f32", 8192, 300)]
 
 
-def _row_kernel_or_skip(B, Hkv, n_vis):
-    if cq.cq_decode_kernel_name(cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V, B, 4 * Hkv, Hkv, n_vis, 128, 1) != "k_decode_row":
-        pytest.skip("this device has more SMs than rows: the row kernel is not chosen")
+def _check_row_kernel(B, Hkv, n_vis):
+    assert cq.cq_decode_kernel_name(cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V, B, 4 * Hkv, Hkv, n_vis, 128, 1) == "k_decode_row"
 
 
 @pytest.mark.parametrize("dtype,n_vis,n_text", ROW_CASES)
-def test_mixed_through_the_row_kernel(cuda_device, dtype, n_vis, n_text):
-    """Enough (sequence, kv-head) rows for the one-CTA-per-row kernel, which
-    attends the text tokens in the same launch (f16: through the ring and the
+def test_mixed_through_the_row_kernel(row_kernel, dtype, n_vis, n_text):
+    """The one-CTA-per-row kernel (forced), which attends the text tokens in
+    the same launch (f16: through the ring and the
     tensor cores, 64 tokens per chunk, whole and partial chunks, odd and even
     chunk-pair counts; f32: on the CUDA cores); and equality with the plain
     decode without text."""
     B, Hkv = 38, 4  # 152 rows: at least one per SM
-    _row_kernel_or_skip(B, Hkv, n_vis)
+    cuda_device = row_kernel
+    _check_row_kernel(B, Hkv, n_vis)
     q, k, v, kt, vt = _case(B, Hkv, n_vis, n_text, dtype, 1, seed=77 + n_vis + n_text)
     qd = q.to(cuda_device)
     kq = cq.cq_quantize_kv(k.to(cuda_device), 1, cq.LAYOUT_OCTET_K)
@@ -97,12 +97,13 @@ def test_mixed_through_the_row_kernel(cuda_device, dtype, n_vis, n_text):
 
 
 @pytest.mark.parametrize("text_scale", [0.05, 4.0])
-def test_row_kernel_text_logits_far_from_visual(cuda_device, text_scale):
+def test_row_kernel_text_logits_far_from_visual(row_kernel, text_scale):
     """Text keys scaled so that the text logits sit well inside (0.05) or far
     above (4.0) the visual ones: the log-sum-exp merge has to keep whichever
     side carries the weight."""
     B, Hkv = 38, 4
-    _row_kernel_or_skip(B, Hkv, 1500)
+    cuda_device = row_kernel
+    _check_row_kernel(B, Hkv, 1500)
     q, k, v, kt, vt = _case(B, Hkv, 1500, 200, "f16", 1, seed=31)
     kt = (kt.double() * text_scale).to(torch.float16)
     qd = q.to(cuda_device)

@@ -1,8 +1,9 @@
-"""GPU parity of the one-CTA-per-row 1-bit decode kernel (chosen when every
-SM gets a (batch, kv-head) row) against the fp64 oracle: calibration
+"""GPU parity of the one-CTA-per-row 1-bit decode kernel against the fp64
+oracle: calibration
 variants in both dtypes, the degenerate cases of the method (all logits
-equal, constant channels, a single token) and determinism. 38 sequences x 4
-kv-heads = 152 rows; each test checks that the row kernel is the one chosen."""
+equal, constant channels, a single token) and determinism. The kernel is
+forced (cq_set_decode_kernel) and each test checks that it is the one
+launched; 38 sequences x 4 kv-heads = 152 rows."""
 
 import pytest
 import torch
@@ -19,10 +20,8 @@ B, HKV = 38, 4
 CALIBS = [(False, 1.0, 1.0), (True, 0.8, 0.9), (True, 1.0, 0.5), (True, 0.5, 1.0)]
 
 
-def _row_kernel_or_skip(n):
-    name = cq.cq_decode_kernel_name(cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V, B, 4 * HKV, HKV, n, 128, 1)
-    if name != "k_decode_row":
-        pytest.skip(f"{name} is chosen on this device (more SMs than rows)")
+def _check_row_kernel(n):
+    assert cq.cq_decode_kernel_name(cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V, B, 4 * HKV, HKV, n, 128, 1) == "k_decode_row"
 
 
 def _quant(k, v, device):
@@ -38,59 +37,59 @@ def _err(out, q, k, v, calib):
 
 @pytest.mark.parametrize("calib", CALIBS)
 @pytest.mark.parametrize("dtype", ["f16", "f32"])
-def test_row_kernel_calibrations_and_dtypes(cuda_device, calib, dtype):
+def test_row_kernel_calibrations_and_dtypes(row_kernel, calib, dtype):
     n = 1000  # four 256-token tiles, the last one ragged
-    _row_kernel_or_skip(n)
+    _check_row_kernel(n)
     q, k, v = synth.make_case(B, 4 * HKV, HKV, n, 128, dtype, outliers=4, seed=101)
-    kq, vq = _quant(k, v, cuda_device)
-    out = cq.cq_decode_attn(q.to(cuda_device), kq, vq, calib=calib)
+    kq, vq = _quant(k, v, row_kernel)
+    out = cq.cq_decode_attn(q.to(row_kernel), kq, vq, calib=calib)
     torch.cuda.synchronize()
     assert _err(out, q, k, v, calib) <= OUT_RTOL
 
 
-def test_row_kernel_equal_logits(cuda_device):
+def test_row_kernel_equal_logits(row_kernel):
     """Zero query: every logit is the same, the range is empty (M = m), the
     calibration leaves it as is and the weights are uniform."""
     n = 600
-    _row_kernel_or_skip(n)
+    _check_row_kernel(n)
     q, k, v = synth.make_case(B, 4 * HKV, HKV, n, 128, "f16", seed=5)
     q.zero_()
-    kq, vq = _quant(k, v, cuda_device)
+    kq, vq = _quant(k, v, row_kernel)
     for calib in CALIBS[:2]:
-        out = cq.cq_decode_attn(q.to(cuda_device), kq, vq, calib=calib)
+        out = cq.cq_decode_attn(q.to(row_kernel), kq, vq, calib=calib)
         torch.cuda.synchronize()
         assert _err(out, q, k, v, calib) <= OUT_RTOL
 
 
-def test_row_kernel_constant_channels(cuda_device):
+def test_row_kernel_constant_channels(row_kernel):
     """beta == alpha in every channel: codes are 0, the step is 0, and the
     output is the constant value exactly."""
     n = 300
-    _row_kernel_or_skip(n)
+    _check_row_kernel(n)
     k = torch.full((B, HKV, n, 128), 1.5, dtype=torch.float16)
     v = torch.full((B, HKV, n, 128), -0.75, dtype=torch.float16)
     q = torch.randn(B, 4 * HKV, 128, generator=torch.Generator().manual_seed(3)).half()
-    kq, vq = _quant(k, v, cuda_device)
-    out = cq.cq_decode_attn(q.to(cuda_device), kq, vq, calib=CALIBS[1]).cpu()
+    kq, vq = _quant(k, v, row_kernel)
+    out = cq.cq_decode_attn(q.to(row_kernel), kq, vq, calib=CALIBS[1]).cpu()
     assert torch.all(out == -0.75)
 
 
-def test_row_kernel_single_token(cuda_device):
+def test_row_kernel_single_token(row_kernel):
     """One token: its weight is 1 and the output is its value, which a 1-bit
     code with alpha = beta = x reproduces exactly."""
-    _row_kernel_or_skip(1)
+    _check_row_kernel(1)
     q, k, v = synth.make_case(B, 4 * HKV, HKV, 1, 128, "f16", seed=6)
-    kq, vq = _quant(k, v, cuda_device)
-    out = cq.cq_decode_attn(q.to(cuda_device), kq, vq, calib=CALIBS[1]).cpu()
+    kq, vq = _quant(k, v, row_kernel)
+    out = cq.cq_decode_attn(q.to(row_kernel), kq, vq, calib=CALIBS[1]).cpu()
     assert torch.equal(out, v[:, :, 0, :].repeat_interleave(4, dim=1))
 
 
-def test_row_kernel_deterministic(cuda_device):
+def test_row_kernel_deterministic(row_kernel):
     n = 3000
-    _row_kernel_or_skip(n)
+    _check_row_kernel(n)
     q, k, v = synth.make_case(B, 4 * HKV, HKV, n, 128, "f16", seed=9)
-    kq, vq = _quant(k, v, cuda_device)
-    qd = q.to(cuda_device)
+    kq, vq = _quant(k, v, row_kernel)
+    qd = q.to(row_kernel)
     o1 = cq.cq_decode_attn(qd, kq, vq, calib=CALIBS[1]).clone()
     for _ in range(3):
         o2 = cq.cq_decode_attn(qd, kq, vq, calib=CALIBS[1])
