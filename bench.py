@@ -216,11 +216,10 @@ def run_ours(args, world, rank, local):
         k_text = synth.make_cache(B, w.hkv, n_text, w.d, w.dtype, 0, gt, device)
         v_text = synth.make_cache(B, w.hkv, n_text, w.d, w.dtype, 0, gt, device)
         dws = torch.empty(cq.cq_decode_attn_mixed_workspace_size(B, w.hq, w.d), dtype=torch.uint8, device=device)
-        launches_per_step = 2
     else:
         dws_n = cq.cq_decode_attn_workspace_size(layouts[0], layouts[1], B, w.hq, w.hkv, n, w.d, bits)
         dws = torch.empty(dws_n, dtype=torch.uint8, device=device) if dws_n else None
-        launches_per_step = 1 if args.path == "octet" else 3
+    launches_per_step = cq.cq_decode_launch_count(layouts[0], layouts[1], B, w.hq, w.hkv, n, w.d, bits, n_text)
 
     def decode(qq):
         if n_text:
@@ -336,7 +335,9 @@ def run_ours(args, world, rank, local):
                      "traffic": None if trec is None else trec["dram_bytes_per_launch"],
                      "algorithmic_bytes_per_launch": alg,
                      "kernel": kernel + ((" (text tokens in the same launch)" if kernel == "k_decode_row"
-                                          else " (partial) + k_text_merge_mma") if n_text else "")},
+                                          else " (partial) + k_text_merge_mma") if n_text else
+                                         (" + split-row launch (2-CTA clusters)"
+                                          if kernel == "k_decode_row" and launches_per_step == 2 else ""))},
         "cache_fill": {"ms": fill_mean, "algorithmic_bytes": fill_alg,
                        "achieved_gbs": fill_alg / (fill_mean * 1e-3) / 1e9,
                        "frac": fill_alg / (fill_mean * 1e-3) / 1e9 / peak},

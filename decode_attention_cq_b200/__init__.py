@@ -25,6 +25,7 @@ from .calibq import (  # noqa: F401
     cq_decode_attn_mixed_workspace_size,
     cq_decode_attn_workspace_size,
     cq_decode_kernel_name,
+    cq_decode_launch_count,
     cq_set_decode_kernel,
     cq_dequant,
     cq_quantize_kv,

@@ -34,6 +34,7 @@ ENTRY_POINTS = (
     "cq_decode_attn_workspace_size",
     "cq_decode_kernel_name",
     "cq_set_decode_kernel",
+    "cq_decode_launch_count",
     "cq_decode_attn",
     "cq_decode_attn_mixed_workspace_size",
     "cq_decode_attn_mixed",
@@ -62,6 +63,7 @@ _SIGS = {
     "cq_decode_attn_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "cq_decode_kernel_name": ([_I, _I, _I, _I, _I, _I, _I, _I], ctypes.c_char_p),
     "cq_set_decode_kernel": ([_I], _I),
+    "cq_decode_launch_count": ([_I, _I, _I, _I, _I, _I, _I, _I, _I], _I),
     "cq_decode_attn": ([_P, _I, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F,
                         cq_calib, _P, _P, _SZ, _P], _I),
     "cq_decode_attn_mixed_workspace_size": ([_I, _I, _I, ctypes.POINTER(_SZ)], _I),
@@ -215,6 +217,13 @@ def cq_decode_kernel_name(k_layout: int, v_layout: int, B: int, Hq: int, Hkv: in
     """Name of the kernel cq_decode_attn launches for these arguments, or None."""
     name = load().cq_decode_kernel_name(k_layout, v_layout, B, Hq, Hkv, n, d, bits)
     return None if name is None else name.decode()
+
+
+def cq_decode_launch_count(k_layout: int, v_layout: int, B: int, Hq: int, Hkv: int, n: int, d: int,
+                           bits: int, n_text: int = 0) -> int:
+    """Kernel launches of one cq_decode_attn (n_text = 0) or cq_decode_attn_mixed
+    call for these arguments (0: none)."""
+    return load().cq_decode_launch_count(k_layout, v_layout, B, Hq, Hkv, n, d, bits, n_text)
 
 
 def cq_set_decode_kernel(which: int) -> None:

@@ -274,6 +274,22 @@ const char* cq_decode_kernel_name(cq_layout k_layout, cq_layout v_layout, int B,
   }
 }
 
+int cq_decode_launch_count(cq_layout k_layout, cq_layout v_layout, int B, int Hq, int Hkv, int n, int d, int bits,
+                           int n_text) {
+  if (n_text < 0) return 0;
+  const char* name = cq_decode_kernel_name(k_layout, v_layout, B, Hq, Hkv, n, d, bits);
+  if (name == nullptr) return 0;
+  if (k_layout == CQ_LAYOUT_CANONICAL) return n_text > 0 ? 0 : 3;  // mixed calls take the octet layouts only
+  if (bits != 1) return n_text > 0 ? 2 : 1;                          // ring kernel (partial), text merge
+  if (n_text > 0) {  // the row kernel attends the text tokens itself; the others hand over to the text merge
+    if (n > 32768) return 0;
+    return choose_1bit(n, B * Hkv, true) == Kernel1::kRow ? 1 : 2;
+  }
+  if (choose_1bit(n, B * Hkv, false) == Kernel1::kRow)
+    return 1 + (cq::decode_row_split_rows(B * Hkv, n, true) > 0 ? 1 : 0);
+  return 1;
+}
+
 cq_status cq_set_decode_kernel(cq_decode_kernel which) {
   switch (which) {
     case CQ_KERNEL_AUTO: g_set_kernel.store((int)Kernel1::kAuto); return CQ_OK;

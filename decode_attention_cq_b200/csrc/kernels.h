@@ -75,6 +75,9 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cq_dtype dt, cudaStream_t str
 // One CTA per (batch, kv-head) row with the logits in tensor memory (1 bit,
 // octet layouts, Hq = 4 Hkv, n <= 8192).
 bool decode_row_supports(int n);
+// Rows of a plain decode (no text tokens, no partial result) that the row
+// kernel runs as halves on 2-CTA clusters in a second launch (0: none).
+int decode_row_split_rows(int rows, int n, bool plain);
 cudaError_t launch_decode_row(const DecodeArgs& a, cq_dtype dt, cudaStream_t stream);
 
 }  // namespace cq

@@ -232,6 +232,21 @@ cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, con
 const char* cq_decode_kernel_name(cq_layout k_layout, cq_layout v_layout, int B, int Hq, int Hkv, int n, int d,
                                   int bits);
 
+/*
+ * Number of kernel launches that cq_decode_attn (n_text = 0) or
+ * cq_decode_attn_mixed (n_text > 0 text tokens) makes for these arguments on
+ * the current device, or 0 when the call would launch none. Host-only.
+ *   canonical layouts: 3; octet layouts: 1 per call, except that a mixed
+ *   call hands the text tokens to a second kernel unless the row kernel takes
+ *   them, and that a plain 1-bit call on the row kernel with more than two
+ *   waves of rows (two rows per SM) runs the rows beyond a whole number of SM
+ *   counts, when they are at most half the SM count, as half rows on 2-CTA
+ *   clusters, in a second launch on a side stream forked from and joined back
+ *   into `stream`.
+ */
+int cq_decode_launch_count(cq_layout k_layout, cq_layout v_layout, int B, int Hq, int Hkv, int n, int d, int bits,
+                           int n_text);
+
 /* 1-bit octet-layout decode kernels, for cq_set_decode_kernel. */
 typedef enum cq_decode_kernel {
   CQ_KERNEL_ENV = -1,     /* CALIBQ_DECODE_KERNEL decides, else the estimate (the initial state) */

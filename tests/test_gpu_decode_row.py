@@ -95,3 +95,27 @@ def test_row_kernel_deterministic(row_kernel):
         o2 = cq.cq_decode_attn(qd, kq, vq, calib=CALIBS[1])
     torch.cuda.synchronize()
     assert torch.equal(o1, o2)
+
+
+@pytest.mark.parametrize("n", [8192, 3000, 257])
+def test_row_kernel_split_rows(row_kernel, n):
+    """More than two waves of rows (two per SM): the rows beyond a whole number
+    of SM counts run as halves on 2-CTA clusters, in a second launch. Every
+    such row, and whole rows around them, against the oracle."""
+    Bb, Hkv = 40, 8  # 320 rows
+    rows = Bb * Hkv
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    split = rows % sms if rows > 2 * sms and (n + 255) // 256 >= 2 and rows % sms <= sms // 2 else 0
+    K, V = cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V
+    assert cq.cq_decode_launch_count(K, V, Bb, 4 * Hkv, Hkv, n, 128, 1) == (2 if split else 1)
+    q, k, v = synth.make_case(Bb, 4 * Hkv, Hkv, n, 128, "f16", outliers=4, seed=n + 13)
+    kq, vq = _quant(k, v, row_kernel)
+    calib = CALIBS[1]
+    out = cq.cq_decode_attn(q.to(row_kernel), kq, vq, calib=calib).cpu()
+    first_split_batch = (rows - split) // Hkv
+    batches = sorted({0, Bb // 2, max(0, first_split_batch - 1)} | set(range(first_split_batch, Bb)))
+    for b in batches:
+        sl = slice(b, b + 1)
+        ref = oracle.decode_attention(f64(q[sl]), f64(k[sl]), f64(v[sl]), 1, "f16", calib)["out"]
+        err = row_rel_err(out[sl].float().numpy(), ref_output_rounded(ref, torch.float16))
+        assert err <= OUT_RTOL, (n, b, err)
