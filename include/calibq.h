@@ -199,7 +199,8 @@ cq_status cq_decode_attn_workspace_size(cq_layout k_layout, cq_layout v_layout, 
  *
  * Supported layout pairs: (CANONICAL, CANONICAL) for any bits and any Hq/Hkv;
  * (OCTET_K, OCTET_V) for d = 128, Hq = 4*Hkv and n <= 65536 at bits = 1
- * (n <= 32768 at bits 2, 4, 8) -- the tensor-core path, one launch per call.
+ * (n <= 32768 at bits 2, 4, 8) -- the tensor-core path, one launch per call
+ * (two for some batches of the 1-bit row kernel: cq_decode_launch_count).
  * cq_decode_kernel_name says which kernel a call launches; the 1-bit kernels
  * agree with each other within the output tolerance, not bit for bit.
  */
