@@ -47,7 +47,9 @@
 //     masked to bit k. Sum_l 2^(8l-31) D_l = sum c p;
 //  7. the four warp pairs' sums meet in shared memory; o = alpha_V + s_V (.)
 //     sum c p / sum p.
-// One launch per decode step, no workspace; n <= 8192 tokens per row.
+// No workspace; n <= 8192 tokens per row. One launch per decode step, plus,
+// past two full waves of rows, a second one that splits the rows beyond a
+// whole number of SM counts over 2-CTA clusters (decode_row_split_rows).
 #include <float.h>
 
 #include <type_traits>
