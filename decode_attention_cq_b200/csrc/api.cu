@@ -84,30 +84,35 @@ int sm_count() {
 // 8192 over 128 to 512 rows (every point within about 3 us). The row kernel
 // runs two CTAs per SM: t1 is a row alone on its SM, t2 a wave of two per SM,
 // and a partial last wave costs 0.6 t1 when it leaves at most one row per SM,
-// else 0.8 t2. The cluster kernel's time grows about linearly in the rows.
-double est_row_us(int n, long long rows, int sms) {
+// else 0.8 t2; a plain decode whose leftover rows run as split halves
+// (decode_row_split_rows) gains about 0.1 t2. The cluster kernel's time grows
+// about linearly in the rows.
+double est_row_us(int n, long long rows, int sms, bool split) {
   const double t1 = 12.8 + 0.00243 * n, t2 = 16.7 + 0.0037 * n;
   if (rows <= sms) return t1;
   const long long slots = 2LL * sms, full = rows / slots, rest = rows % slots;
   if (full == 0) return t2;
-  return (double)full * t2 + (rest == 0 ? 0.0 : rest <= sms ? 0.6 * t1 : 0.8 * t2);
+  return (double)full * t2 + (rest == 0 ? 0.0 : rest <= sms ? 0.6 * t1 : 0.8 * t2) - (split ? 0.1 * t2 : 0.0);
 }
 double est_cluster_us(int n, long long rows) { return 11.7 + (double)rows * (0.0065 + 1.77e-5 * n); }
 
-Kernel1 choose_1bit(int n, int rows, bool partial) {
+// partial: the visual part of a two-launch mixed call (no tcgen05 kernel);
+// plain: a decode with no text tokens and no partial result (rows may split).
+Kernel1 choose_1bit(int n, int rows, bool partial, bool plain) {
   const Kernel1 f = forced_kernel();
   if (f == Kernel1::kRow && cq::decode_row_supports(n)) return Kernel1::kRow;
   if (f == Kernel1::kCluster && cq::decode_mma_supports(n)) return Kernel1::kCluster;
   if (f == Kernel1::kTcgen05 && !partial) return Kernel1::kTcgen05;
   const int sms = sm_count();
-  if (cq::decode_row_supports(n) && sms > 0 && est_row_us(n, rows, sms) < est_cluster_us(n, rows))
+  const bool split = plain && cq::decode_row_split_rows(rows, n, true) > 0;
+  if (cq::decode_row_supports(n) && sms > 0 && est_row_us(n, rows, sms, split) < est_cluster_us(n, rows))
     return Kernel1::kRow;
   if (cq::decode_mma_supports(n)) return Kernel1::kCluster;
   return partial ? Kernel1::kAuto : Kernel1::kTcgen05;  // kAuto: none
 }
 
 cudaError_t launch_decode_1bit(const cq::DecodeArgs& a, cq_dtype dt, cudaStream_t s) {
-  switch (choose_1bit(a.n, a.B * a.Hkv, a.part_o != nullptr)) {
+  switch (choose_1bit(a.n, a.B * a.Hkv, a.part_o != nullptr, a.part_o == nullptr && a.n_text == 0)) {
     case Kernel1::kRow: return cq::launch_decode_row(a, dt, s);
     case Kernel1::kCluster: return cq::launch_decode_mma(a, dt, s);
     case Kernel1::kTcgen05: return cq::launch_decode_octet(a, dt, s);
@@ -267,7 +272,7 @@ const char* cq_decode_kernel_name(cq_layout k_layout, cq_layout v_layout, int B,
   if (k_layout != CQ_LAYOUT_OCTET_K || v_layout != CQ_LAYOUT_OCTET_V || G != 4) return nullptr;
   if (bits != 1) return cq::decode_ring_supports(n, bits) ? "k_decode_ring" : nullptr;
   if (n > 65536) return nullptr;
-  switch (choose_1bit(n, B * Hkv, false)) {
+  switch (choose_1bit(n, B * Hkv, false, true)) {
     case Kernel1::kRow: return "k_decode_row";
     case Kernel1::kCluster: return "k_decode_mma";
     default: return "k_decode_octet";
@@ -283,9 +288,9 @@ int cq_decode_launch_count(cq_layout k_layout, cq_layout v_layout, int B, int Hq
   if (bits != 1) return n_text > 0 ? 2 : 1;                          // ring kernel (partial), text merge
   if (n_text > 0) {  // the row kernel attends the text tokens itself; the others hand over to the text merge
     if (n > 32768) return 0;
-    return choose_1bit(n, B * Hkv, true) == Kernel1::kRow ? 1 : 2;
+    return choose_1bit(n, B * Hkv, false, false) == Kernel1::kRow ? 1 : 2;
   }
-  if (choose_1bit(n, B * Hkv, false) == Kernel1::kRow)
+  if (choose_1bit(n, B * Hkv, false, true) == Kernel1::kRow)
     return 1 + (cq::decode_row_split_rows(B * Hkv, n, true) > 0 ? 1 : 0);
   return 1;
 }
@@ -372,7 +377,7 @@ cq_status cq_decode_attn_mixed(const void* q, cq_dtype dt, const uint8_t* k_code
   cq::DecodeArgs a = make_args(q, k_codes, k_alpha, k_scale, v_codes, v_alpha, v_scale, B, Hq, Hkv, n_vis, d,
                                bits, softmax_scale, calib, out);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (bits == 1 && choose_1bit(n_vis, B * Hkv, false) == Kernel1::kRow) {
+  if (bits == 1 && choose_1bit(n_vis, B * Hkv, false, false) == Kernel1::kRow) {
     // one launch: the row kernel attends the text tokens after the quantized ones
     a.k_text = k_text;
     a.v_text = v_text;
