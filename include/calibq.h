@@ -243,7 +243,10 @@ const char* cq_decode_kernel_name(cq_layout k_layout, cq_layout v_layout, int B,
  *   waves of rows (two rows per SM) runs the rows beyond a whole number of SM
  *   counts, when they are at most half the SM count, as half rows on 2-CTA
  *   clusters, in a second launch on a side stream forked from and joined back
- *   into `stream`.
+ *   into `stream`. That side stream and its two events are created once per
+ *   host thread and device, by the first such call; make that call outside
+ *   stream capture (a warm-up call before capturing a CUDA graph), since a
+ *   capture in the global mode does not allow creating them.
  */
 int cq_decode_launch_count(cq_layout k_layout, cq_layout v_layout, int B, int Hq, int Hkv, int n, int d, int bits,
                            int n_text);
