@@ -20,7 +20,6 @@ bool valid_dtype(cq_dtype dt) { return dt == CQ_F16 || dt == CQ_F32; }
 bool valid_layout(cq_layout l) {
   return l == CQ_LAYOUT_CANONICAL || l == CQ_LAYOUT_OCTET_K || l == CQ_LAYOUT_OCTET_V;
 }
-size_t dsize(cq_dtype dt) { return dt == CQ_F16 ? 2 : 4; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Device memory of the current device (or managed memory) and 16-byte aligned.
