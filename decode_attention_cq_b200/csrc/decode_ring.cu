@@ -171,15 +171,27 @@ __global__ void __launch_bounds__(kThreads, ring_slots<BITS>() == 2 ? 3 : 2)
     const int ch = t & (kD - 1);
     const float ak = DT<T>::f(sRows[4 * kD + ch]);
     const float sk = DT<T>::f(sRows[5 * kD + ch]);
+    float amax[kG], qa[kG];
 #pragma unroll
     for (int h = 0; h < kG; ++h) {
       const float qv = DT<T>::f(sRows[h * kD + ch]);
       w[h] = a.sigma * qv * sk;
-      const float amax = warp_max(fabsf(w[h]));
-      const float qa = warp_sum(qv * ak);
-      if (lane == 0 && warp < kD / 32) {
-        F.red[warp][h][0] = amax;
-        F.red[warp][h][1] = qa;
+      amax[h] = fabsf(w[h]);
+      qa[h] = qv * ak;
+    }
+    // the four heads' reductions interleaved, with no branch between them
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+#pragma unroll
+      for (int h = 0; h < kG; ++h) {
+        amax[h] = fmaxf(amax[h], __shfl_xor_sync(0xffffffffu, amax[h], o));
+        qa[h] += __shfl_xor_sync(0xffffffffu, qa[h], o);
+      }
+    if (lane == 0 && warp < kD / 32) {
+#pragma unroll
+      for (int h = 0; h < kG; ++h) {
+        F.red[warp][h][0] = amax[h];
+        F.red[warp][h][1] = qa[h];
       }
     }
   }
@@ -188,8 +200,8 @@ __global__ void __launch_bounds__(kThreads, ring_slots<BITS>() == 2 ? 3 : 2)
 #pragma unroll
     for (int h = 0; h < kG; ++h) {
       const float amax = fmaxf(fmaxf(F.red[0][h][0], F.red[1][h][0]), fmaxf(F.red[2][h][0], F.red[3][h][0]));
-      const float ks = amax > 0.f ? amax / (float)kWMax : 0.f;
-      const float inv = ks > 0.f ? 1.f / ks : 0.f;
+      const float ks = amax * (1.f / (float)kWMax);              // any scale works: w is rounded with this one
+      const float inv = ks > 0.f ? __fdividef(1.f, ks) : 0.f;  // approximate: the clamp below bounds w
       const int wi = max(-kWMax, min(kWMax, __float2int_rn(w[h] * inv)));
       F.limb[3 * h + 0][t] = (uint8_t)(wi & 127);
       F.limb[3 * h + 1][t] = (uint8_t)((wi >> 7) & 127);
