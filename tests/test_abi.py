@@ -113,6 +113,25 @@ def test_set_decode_kernel_forces_and_releases(lib):
         cq.cq_set_decode_kernel(cq.KERNEL_ENV)
 
 
+def test_decode_launch_count(lib):
+    K, V, C = cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V, cq.LAYOUT_CANONICAL
+    assert cq.cq_decode_launch_count(C, C, 2, 8, 2, 1000, 128, 2) == 3  # scores, softmax-V, merge
+    assert cq.cq_decode_launch_count(C, C, 2, 8, 2, 1000, 128, 2, 16) == 0  # mixed calls take octet layouts
+    assert cq.cq_decode_launch_count(K, V, 2, 8, 2, 1000, 128, 2) == 1
+    assert cq.cq_decode_launch_count(K, V, 2, 8, 2, 1000, 128, 2, 16) == 2  # ring kernel, then the text merge
+    assert cq.cq_decode_launch_count(K, V, 2, 8, 2, 1000, 64, 1) == 0  # unsupported d
+    assert cq.cq_decode_launch_count(K, V, 2, 8, 2, 1000, 128, 1, -1) == 0
+    try:
+        cq.cq_set_decode_kernel(cq.KERNEL_ROW)
+        assert cq.cq_decode_launch_count(K, V, 2, 8, 2, 1000, 128, 1, 16) == 1  # text in the same launch
+        cq.cq_set_decode_kernel(cq.KERNEL_CLUSTER)
+        assert cq.cq_decode_launch_count(K, V, 2, 8, 2, 1000, 128, 1) == 1
+        assert cq.cq_decode_launch_count(K, V, 2, 8, 2, 1000, 128, 1, 16) == 2
+        assert cq.cq_decode_launch_count(K, V, 2, 8, 2, 40000, 128, 1, 16) == 0  # mixed: n <= 32768
+    finally:
+        cq.cq_set_decode_kernel(cq.KERNEL_ENV)
+
+
 def test_null_pointers_rejected_before_any_cuda_call(lib):
     st = lib.cq_quantize_kv(None, 0, 1, 1, 16, 128, 1, 0, None, None, None, None, 0, None)
     assert st == cq.CQ_ERR_INVALID_ARG
