@@ -16,7 +16,8 @@
 // per SM), written and read back by the thread that owns them.
 //
 // Tiles of 256 tokens (32 octets), 8 warps, two CTAs per SM:
-//  1. one thread copies the q / alpha / s rows and the first chunks of codes;
+//  1. one thread copies the q / alpha / s rows and the first chunks of codes
+//     while warp 0 allocates tensor memory;
 //     the K codes and after them the V codes stream through a ring of 16 KB
 //     slots (4 tiles each; tensor copies with the 128-byte swizzle, completing
 //     on a full mbarrier per slot, every wait bounded). A shared counter per
@@ -40,13 +41,17 @@
 //  5. each lane turns its 32 logit columns of a tile, in place, into its A-fragment
 //     words of the tile's 8 bit positions for the V side: P = p 2^(31-k) for its
 //     own bit of every pair, a swap with lane ^ 16, byte permutes into limb rows
-//     (rows 4 limb + head, columns octets);
+//     (rows 4 limb + head, columns octets); each warp of a pair forms half of
+//     the bit positions of the pair's next tile while it issues the current
+//     tile's V MMAs, and a 64-thread barrier per tile hands the halves over;
 //  6. V side: warp pair (q, q + 4) (the two warps sharing a tensor-memory lane
 //     quarter) takes tiles q, q + 4, ... and splits the 128 channels; A = the
 //     tile's fragments loaded from tensor memory, B = V codes of 8 channels
 //     masked to bit k. Sum_l 2^(8l-31) D_l = sum c p;
 //  7. the four warp pairs' sums meet in shared memory; o = alpha_V + s_V (.)
-//     sum c p / sum p.
+//     sum c p / sum p; with text tokens (a mixed cache) the warps first attend
+//     them (f16: through the ring and the tensor cores) and the output merges
+//     both parts by their log-sum-exps.
 // No workspace; n <= 8192 tokens per row. One launch per decode step, plus,
 // past two full waves of rows, a second one that splits the rows beyond a
 // whole number of SM counts over 2-CTA clusters (decode_row_split_rows).
