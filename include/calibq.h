@@ -11,8 +11,12 @@
  *
  *  - All tensor pointers are DEVICE pointers owned by the caller (device or
  *    managed memory of the current device; host pointers are rejected with
- *    CQ_ERR_INVALID_ARG). The library never allocates in these calls and keeps
- *    no mutable global state; calls are thread-safe.
+ *    CQ_ERR_INVALID_ARG). The library never allocates device memory in these
+ *    calls. Host-side state: the kernel choice set by cq_set_decode_kernel
+ *    (process-wide), a small cache of encoded tensor maps per host thread,
+ *    and per host thread and device one stream and two events, created by the
+ *    first decode that splits rows (cq_decode_launch_count). Calls are
+ *    thread-safe.
  *  - Work is enqueued asynchronously on `stream` (NULL = the legacy default
  *    stream). A returned CQ_OK means the launch was enqueued; kernel faults
  *    surface on the stream like any CUDA error.
