@@ -53,3 +53,22 @@ def test_two_gloo_ranks_agree_on_max_and_reference_runs_on_rank0():
     assert [r[1] for r in res] == [2.5, 2.5]  # max over ranks, seen by both
     assert res[0][2] == ("reference", 2, True)
     assert res[1][2] is None
+
+
+def test_reference_line_keeps_the_contract():
+    """The reference arm's JSON line (one process, the tiny workload): the base
+    keys, the oracle as its own CPU baseline, and an end-to-end figure equal to
+    its value with no host-device copies."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    args = types.SimpleNamespace(workload="tiny_n256", steps=1, warmup=3)
+    line = bench.run_reference(args, 1, 0)
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["n_gpus"] == 1 and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["cores"] >= 1 and line["cpu_baseline"]["sample"]
+    assert line["e2e"]["value"] == line["value"] and line["e2e"]["unit"] == line["unit"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
