@@ -39,7 +39,7 @@ METRIC = "1-bit decode-attention tokens/s and achieved HBM GB/s (n=8192), % of r
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 FALLBACK_HBM_GBS = 6650.0
 CALIB = (True, 0.8, 0.9)
-KERNEL_SOURCES = {"k_decode_row": "decode_row.cu", "k_decode_mma": "decode_mma.cu",
+KERNEL_SOURCES = {"k_decode_tc": "decode_tc.cu", "k_decode_row": "decode_row.cu", "k_decode_mma": "decode_mma.cu",
                   "k_decode_octet": "decode_octet.cu", "k_decode_ring": "decode_ring.cu",
                   "k_scores + k_softmax_v + k_merge": "decode_generic.cu"}
 

@@ -15,6 +15,7 @@ from .calibq import (  # noqa: F401
     KERNEL_AUTO,
     KERNEL_CLUSTER,
     KERNEL_ENV,
+    KERNEL_PIPE,
     KERNEL_ROW,
     KERNEL_TCGEN05,
     CalibqError,

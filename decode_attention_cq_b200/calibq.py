@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libc
 CQ_OK, CQ_ERR_INVALID_ARG, CQ_ERR_UNSUPPORTED, CQ_ERR_WORKSPACE, CQ_ERR_CUDA = range(5)
 CQ_F16, CQ_F32 = 0, 1
 LAYOUT_CANONICAL, LAYOUT_OCTET_K, LAYOUT_OCTET_V = 0, 1, 2
-KERNEL_ENV, KERNEL_AUTO, KERNEL_ROW, KERNEL_CLUSTER, KERNEL_TCGEN05 = -1, 0, 1, 2, 3
+KERNEL_ENV, KERNEL_AUTO, KERNEL_ROW, KERNEL_CLUSTER, KERNEL_TCGEN05, KERNEL_PIPE = -1, 0, 1, 2, 3, 4
 
 ENTRY_POINTS = (
     "cq_version",
@@ -228,7 +228,7 @@ def cq_decode_launch_count(k_layout: int, v_layout: int, B: int, Hq: int, Hkv: i
 
 def cq_set_decode_kernel(which: int) -> None:
     """Force a 1-bit octet decode kernel for the rest of the process
-    (KERNEL_ROW / KERNEL_CLUSTER / KERNEL_TCGEN05), let the estimate decide
+    (KERNEL_PIPE / KERNEL_ROW / KERNEL_CLUSTER / KERNEL_TCGEN05), let the estimate decide
     (KERNEL_AUTO), or go back to the environment (KERNEL_ENV)."""
     _check(load().cq_set_decode_kernel(int(which)), "cq_set_decode_kernel")
 

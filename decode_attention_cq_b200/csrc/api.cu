@@ -40,13 +40,15 @@ cq_status check_ptr(const void* p) {
 }
 
 // 1-bit octet-layout decode kernels: "row" (one CTA per row, logits in tensor
-// memory, n <= 8192), "cluster" (a cluster of CTAs per row, n <= 32768) and
-// "tcgen05" (5th-generation tensor cores, n <= 65536). cq_set_decode_kernel,
-// else the environment variable CALIBQ_DECODE_KERNEL, may name one to use
-// wherever it supports n; otherwise the choice between the row and the cluster
-// kernel is the one with the smaller estimated step time, and the tcgen05
-// kernel takes what neither supports.
-enum class Kernel1 { kAuto, kRow, kCluster, kTcgen05 };
+// memory, n <= 8192), "cluster" (a cluster of CTAs per row, n <= 32768),
+// "tcgen05" (5th-generation tensor cores, n <= 65536) and "pipe" (one
+// persistent CTA per SM whose warps feed tcgen05 MMAs, plain decodes with
+// n <= 8192; measured slower than "row" on B200, so only on request).
+// cq_set_decode_kernel, else the environment variable CALIBQ_DECODE_KERNEL,
+// may name one to use wherever it supports the call; otherwise the choice
+// between the row and the cluster kernel is the one with the smaller
+// estimated step time, and the tcgen05 kernel takes what neither supports.
+enum class Kernel1 { kAuto, kRow, kCluster, kTcgen05, kPipe };
 
 Kernel1 env_kernel() {
   static const Kernel1 forced = [] {
@@ -55,6 +57,7 @@ Kernel1 env_kernel() {
     if (strcmp(v, "row") == 0) return Kernel1::kRow;
     if (strcmp(v, "cluster") == 0) return Kernel1::kCluster;
     if (strcmp(v, "tcgen05") == 0) return Kernel1::kTcgen05;
+    if (strcmp(v, "pipe") == 0) return Kernel1::kPipe;
     return Kernel1::kAuto;
   }();
   return forced;
@@ -99,6 +102,8 @@ double est_cluster_us(int n, long long rows) { return 11.7 + (double)rows * (0.0
 // plain: a decode with no text tokens and no partial result (rows may split).
 Kernel1 choose_1bit(int n, int rows, bool partial, bool plain) {
   const Kernel1 f = forced_kernel();
+  const bool pipe = plain && cq::decode_tc_supports(n);
+  if (f == Kernel1::kPipe && pipe) return Kernel1::kPipe;
   if (f == Kernel1::kRow && cq::decode_row_supports(n)) return Kernel1::kRow;
   if (f == Kernel1::kCluster && cq::decode_mma_supports(n)) return Kernel1::kCluster;
   if (f == Kernel1::kTcgen05 && !partial) return Kernel1::kTcgen05;
@@ -115,6 +120,7 @@ cudaError_t launch_decode_1bit(const cq::DecodeArgs& a, cq_dtype dt, cudaStream_
     case Kernel1::kRow: return cq::launch_decode_row(a, dt, s);
     case Kernel1::kCluster: return cq::launch_decode_mma(a, dt, s);
     case Kernel1::kTcgen05: return cq::launch_decode_octet(a, dt, s);
+    case Kernel1::kPipe: return cq::launch_decode_tc(a, dt, s);
     default: return cudaErrorNotSupported;
   }
 }
@@ -274,6 +280,7 @@ const char* cq_decode_kernel_name(cq_layout k_layout, cq_layout v_layout, int B,
   switch (choose_1bit(n, B * Hkv, false, true)) {
     case Kernel1::kRow: return "k_decode_row";
     case Kernel1::kCluster: return "k_decode_mma";
+    case Kernel1::kPipe: return "k_decode_tc";
     default: return "k_decode_octet";
   }
 }
@@ -300,6 +307,7 @@ cq_status cq_set_decode_kernel(cq_decode_kernel which) {
     case CQ_KERNEL_ROW: g_set_kernel.store((int)Kernel1::kRow); return CQ_OK;
     case CQ_KERNEL_CLUSTER: g_set_kernel.store((int)Kernel1::kCluster); return CQ_OK;
     case CQ_KERNEL_TCGEN05: g_set_kernel.store((int)Kernel1::kTcgen05); return CQ_OK;
+    case CQ_KERNEL_PIPE: g_set_kernel.store((int)Kernel1::kPipe); return CQ_OK;
     case CQ_KERNEL_ENV: g_set_kernel.store(-1); return CQ_OK;
     default: return CQ_ERR_INVALID_ARG;
   }

@@ -80,4 +80,9 @@ bool decode_row_supports(int n);
 int decode_row_split_rows(int rows, int n, bool plain);
 cudaError_t launch_decode_row(const DecodeArgs& a, cq_dtype dt, cudaStream_t stream);
 
+// ---- decode_tc.cu (1 bit, octet layouts, Hq = 4 Hkv, n <= 8192, plain decodes:
+// one persistent CTA per SM, tcgen05 MMAs fed by worker warps, dedicated issuers)
+bool decode_tc_supports(int n);
+cudaError_t launch_decode_tc(const DecodeArgs& a, cq_dtype dt, cudaStream_t stream);
+
 }  // namespace cq

@@ -228,8 +228,11 @@ cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, con
  *     the cluster kernel for short rows and for batches that leave the row
  *     kernel a thin last wave); the tcgen05 kernel takes longer rows.
  *     cq_set_decode_kernel, else the environment variable
- *     CALIBQ_DECODE_KERNEL = row | cluster | tcgen05 (read once per process),
- *     forces one of them wherever it supports n.
+ *     CALIBQ_DECODE_KERNEL = pipe | row | cluster | tcgen05 (read once per process),
+ *     forces one of them wherever it supports n. "k_decode_tc" (pipe: one
+ *     persistent CTA per SM working through whole rows, n <= 8192, plain
+ *     decodes, its warps feeding 5th-generation tensor-core MMAs) is chosen
+ *     only when forced.
  *   2, 4, 8 bits, octet layouts: "k_decode_ring".
  *   Canonical layouts: "k_scores + k_softmax_v + k_merge" (three launches).
  * The returned string is static; the caller does not free it.
@@ -261,7 +264,8 @@ typedef enum cq_decode_kernel {
   CQ_KERNEL_AUTO = 0,     /* the estimate decides, whatever the environment says */
   CQ_KERNEL_ROW = 1,      /* "k_decode_row" wherever n <= 8192 */
   CQ_KERNEL_CLUSTER = 2,  /* "k_decode_mma" wherever n <= 32768 */
-  CQ_KERNEL_TCGEN05 = 3   /* "k_decode_octet" (plain decodes; mixed calls choose as with AUTO) */
+  CQ_KERNEL_TCGEN05 = 3,  /* "k_decode_octet" (plain decodes; mixed calls choose as with AUTO) */
+  CQ_KERNEL_PIPE = 4      /* "k_decode_tc" (plain decodes with n <= 8192; others choose as with AUTO) */
 } cq_decode_kernel;
 
 /*

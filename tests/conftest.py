@@ -36,3 +36,14 @@ def row_kernel(cuda_device):
     cq.cq_set_decode_kernel(cq.KERNEL_ROW)
     yield cuda_device
     cq.cq_set_decode_kernel(cq.KERNEL_ENV)
+
+
+@pytest.fixture
+def pipe_kernel(cuda_device):
+    """Force the persistent tcgen05 1-bit decode kernel (plain decodes with
+    n <= 8192) for one test, then hand the choice back."""
+    from decode_attention_cq_b200 import calibq as cq
+
+    cq.cq_set_decode_kernel(cq.KERNEL_PIPE)
+    yield cuda_device
+    cq.cq_set_decode_kernel(cq.KERNEL_ENV)

@@ -107,8 +107,12 @@ def test_set_decode_kernel_forces_and_releases(lib):
         assert cq.cq_decode_kernel_name(K, V, 1, 8, 2, 32769, 128, 1) == "k_decode_octet"
         cq.cq_set_decode_kernel(cq.KERNEL_TCGEN05)
         assert cq.cq_decode_kernel_name(K, V, 64, 32, 8, 1000, 128, 1) == "k_decode_octet"
+        cq.cq_set_decode_kernel(cq.KERNEL_PIPE)
+        assert cq.cq_decode_kernel_name(K, V, 1, 8, 2, 1000, 128, 1) == "k_decode_tc"
+        assert cq.cq_decode_kernel_name(K, V, 1, 8, 2, 8193, 128, 1) == "k_decode_mma"  # pipe takes n <= 8192
         cq.cq_set_decode_kernel(cq.KERNEL_AUTO)
         assert cq.cq_decode_kernel_name(K, V, 1, 8, 2, 32768, 128, 1) == "k_decode_mma"
+        assert cq.cq_decode_kernel_name(K, V, 64, 32, 8, 8192, 128, 1) in ("k_decode_row", "k_decode_mma")
     finally:
         cq.cq_set_decode_kernel(cq.KERNEL_ENV)
 
@@ -124,6 +128,12 @@ def test_decode_launch_count(lib):
     try:
         cq.cq_set_decode_kernel(cq.KERNEL_ROW)
         assert cq.cq_decode_launch_count(K, V, 2, 8, 2, 1000, 128, 1, 16) == 1  # text in the same launch
+        cq.cq_set_decode_kernel(cq.KERNEL_PIPE)
+        assert cq.cq_decode_launch_count(K, V, 64, 32, 8, 8192, 128, 1) == 1  # one persistent launch
+        cq.cq_set_decode_kernel(cq.KERNEL_AUTO)
+        mixed_auto = cq.cq_decode_launch_count(K, V, 2, 8, 2, 1000, 128, 1, 16)
+        cq.cq_set_decode_kernel(cq.KERNEL_PIPE)
+        assert cq.cq_decode_launch_count(K, V, 2, 8, 2, 1000, 128, 1, 16) == mixed_auto  # mixed: as AUTO
         cq.cq_set_decode_kernel(cq.KERNEL_CLUSTER)
         assert cq.cq_decode_launch_count(K, V, 2, 8, 2, 1000, 128, 1) == 1
         assert cq.cq_decode_launch_count(K, V, 2, 8, 2, 1000, 128, 1, 16) == 2
