@@ -509,6 +509,79 @@ def _time_graph(step, steps: int, warmup: int) -> float:
     return ms
 
 
+def _time_flushed(step, steps: int, warmup: int, flush) -> float:
+    """Mean ms of one step replayed from a CUDA graph, CUDA events on the
+    launching stream around each replay, the L2 flushed (outside the events)
+    before every timed replay."""
+    stream = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for _ in range(warmup):
+            step()
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        step()
+    for it in range(warmup):
+        flush.fill_(it & 255)
+        g.replay()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for it in range(steps):
+        flush.fill_((it * 7) & 255)
+        starts[it].record(stream)
+        g.replay()
+        ends[it].record(stream)
+    torch.cuda.synchronize()
+    del g
+    return sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / steps
+
+
+def run_bit_sweep(args):
+    """Bit-width sweep at bitsweep_n8192_b16 (batch 16, 32 / 8 heads, d = 128,
+    n = 8192, the caches quantized by the library at each b): one JSON line
+    per b in {1, 2, 4, 8} with the step time of one cq_decode_attn call,
+    tokens/s, GB/s of algorithmic bytes and the fraction of the measured copy
+    bandwidth. (The output error of each b against the fp64 oracle is reported
+    by tests/bitsweep_error_report.py on the same seeded inputs.)"""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS["bitsweep_n8192_b16"]
+    q, k, v = synth.make_workload(w, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    peak, peak_src = measured_peaks()
+    K, V = cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V
+    for bits in (1, 2, 4, 8):
+        kq = cq.cq_quantize_kv(k, bits, K)
+        vq = cq.cq_quantize_kv(v, bits, V)
+        out = torch.empty_like(q)
+
+        def step():
+            cq.cq_decode_attn(q, kq, vq, calib=CALIB, out=out)
+
+        ms = _time_flushed(step, min(args.steps, 200), args.warmup, flush)
+        alg = algorithmic_bytes(w.batch, w.hq, w.hkv, w.n, w.d, bits)
+        gbs = alg / (ms * 1e-3) / 1e9
+        print(json.dumps({
+            "metric": "decode-attention tokens/s and achieved HBM GB/s per bit width (n=8192, batch 16)",
+            "bits": bits, "value": w.batch / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "higher_is_better": True, "data": "synthetic (seeded InternVL-2.5-shaped K/V caches)",
+            "config": {"workload": "bitsweep_n8192_b16", "batch": w.batch, "q_heads": w.hq, "kv_heads": w.hkv,
+                       "head_dim": w.d, "n_tokens": w.n, "layout": "octet",
+                       "calibration": {"tau_lo": CALIB[1], "tau_hi": CALIB[2]},
+                       "l2": "flushed (256 MB write) between timed steps"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "peak_source": peak_src, "algorithmic_bytes_per_launch": alg},
+            "kernel": cq.cq_decode_kernel_name(K, V, w.batch, w.hq, w.hkv, w.n, w.d, bits),
+            "gpu_launches_per_step": cq.cq_decode_launch_count(K, V, w.batch, w.hq, w.hkv, w.n, w.d, bits)}),
+            flush=True)
+        del kq, vq, out
+        torch.cuda.empty_cache()
+
+
 def run_budget(args):
     """Memory-budget sweep: a full 32-layer decode step (32 / 8 heads, d = 128,
     n = 3328) with the largest batch whose KV cache fits each budget, 1-bit
@@ -589,12 +662,17 @@ def main():
     ap.add_argument("--budget-sweep", action="store_true",
                     help="32-layer decode step under KV-cache budgets, 1-bit vs f16 cache (one line per budget)")
     ap.add_argument("--budgets", type=float, nargs="+", default=[5, 10, 20, 30])
+    ap.add_argument("--bit-sweep", action="store_true",
+                    help="bit widths 1, 2, 4, 8 at bitsweep_n8192_b16 (one line per width)")
     args = ap.parse_args()
     args_global = args
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.budget_sweep:
         run_budget(args)
+        return
+    if args.bit_sweep:
+        run_bit_sweep(args)
         return
     world, rank, local = dist_setup()
     if args.impl == "reference":

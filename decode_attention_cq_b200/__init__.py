@@ -18,10 +18,12 @@ from .calibq import (  # noqa: F401
     KERNEL_PIPE,
     KERNEL_ROW,
     KERNEL_TCGEN05,
+    DEVICE_WAIT_TIMEOUT,
     CalibqError,
     QuantizedCache,
     cq_codes_bytes,
     cq_decode_attn,
+    cq_decode_attn_ex,
     cq_decode_attn_mixed,
     cq_decode_attn_mixed_workspace_size,
     cq_decode_attn_workspace_size,

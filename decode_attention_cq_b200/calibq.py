@@ -36,6 +36,7 @@ ENTRY_POINTS = (
     "cq_set_decode_kernel",
     "cq_decode_launch_count",
     "cq_decode_attn",
+    "cq_decode_attn_ex",
     "cq_decode_attn_mixed_workspace_size",
     "cq_decode_attn_mixed",
     "cq_dequant",
@@ -66,6 +67,8 @@ _SIGS = {
     "cq_decode_launch_count": ([_I, _I, _I, _I, _I, _I, _I, _I, _I], _I),
     "cq_decode_attn": ([_P, _I, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F,
                         cq_calib, _P, _P, _SZ, _P], _I),
+    "cq_decode_attn_ex": ([_P, _I, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F,
+                           cq_calib, _P, _P, _SZ, _P, ctypes.c_uint, _P], _I),
     "cq_decode_attn_mixed_workspace_size": ([_I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "cq_decode_attn_mixed": ([_P, _I, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _I, _I, _I, _I, _I, _F,
                               cq_calib, _P, _P, _SZ, _P], _I),
@@ -251,6 +254,34 @@ def cq_decode_attn(q: torch.Tensor, k: QuantizedCache, v: QuantizedCache, *,
                                  B, Hq, Hkv, n, d, k.bits, float(softmax_scale), cal, _ptr(out),
                                  _ptr(workspace), 0 if workspace is None else workspace.numel(),
                                  _stream(stream, q)), "cq_decode_attn")
+    return out
+
+
+DEVICE_WAIT_TIMEOUT = 1  # bit of the device status word (CQ_DEVICE_WAIT_TIMEOUT)
+
+
+def cq_decode_attn_ex(q: torch.Tensor, k: QuantizedCache, v: QuantizedCache, status: torch.Tensor, *,
+                      wait_probes: int = 0, calib=(False, 1.0, 1.0), softmax_scale: float = 0.0,
+                      out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    """cq_decode_attn that ORs DEVICE_WAIT_TIMEOUT into `status` (an int32
+    device tensor the caller zeroes) when a kernel's bounded wait ran out;
+    wait_probes > 0 bounds the cluster kernel's copy waits to that many probes."""
+    B, Hq, d = q.shape
+    _, Hkv, n, _ = k.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        ws = cq_decode_attn_workspace_size(k.layout, v.layout, B, Hq, Hkv, n, d, k.bits)
+        workspace = torch.empty(ws, dtype=torch.uint8, device=q.device) if ws else None
+    if status.dtype != torch.int32 or not status.is_cuda:
+        raise ValueError("status must be an int32 CUDA tensor")
+    cal = _calib(bool(calib[0]), float(calib[1]), float(calib[2]))
+    _check(load().cq_decode_attn_ex(_ptr(q), _dt(q), _ptr(k.codes), _ptr(k.alpha), _ptr(k.scale),
+                                    k.layout, _ptr(v.codes), _ptr(v.alpha), _ptr(v.scale), v.layout,
+                                    B, Hq, Hkv, n, d, k.bits, float(softmax_scale), cal, _ptr(out),
+                                    _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                    _ptr(status), int(wait_probes), _stream(stream, q)), "cq_decode_attn_ex")
     return out
 
 

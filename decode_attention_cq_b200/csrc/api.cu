@@ -7,6 +7,7 @@
 #include <limits>
 
 #include "calibq.h"
+#include "common.cuh"
 #include "kernels.h"
 
 namespace {
@@ -70,15 +71,17 @@ Kernel1 forced_kernel() {
   return v < 0 ? env_kernel() : static_cast<Kernel1>(v);
 }
 
+// SM count of the current device (read once per device).
 int sm_count() {
-  static const int count = [] {
-    int dev = 0, c = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) !=
-                                                   cudaSuccess)
-      return 0;
-    return c;
-  }();
-  return count;
+  static std::atomic<int> counts[cq::kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= cq::kMaxDevices) return 0;
+  int c = counts[dev].load(std::memory_order_relaxed);
+  if (c == 0) {
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    counts[dev].store(c, std::memory_order_relaxed);
+  }
+  return c;
 }
 
 // Step-time estimates (microseconds on B200) of the two kernels for `rows`
@@ -239,12 +242,14 @@ cq_status cq_quantize_kv_noalloc(const void* x, cq_dtype dt, int B, int H, int n
   CQ_TRY(check_shape(B, H, n, d, bits));
   size_t rb = 0;
   CQ_TRY(row_bytes(layout, n, bits, &rb));
+  // only the two-launch path (n > 16384) keeps statistics in the scratch
+  if (cq::quantize_uses_workspace(B * H, n) &&
+      cq::quantize_workspace_bytes(B * H, n) > cq::quantize_static_scratch_bytes())
+    return CQ_ERR_UNSUPPORTED;
   CQ_TRY(check_ptr(x));
   CQ_TRY(check_ptr(codes));
   CQ_TRY(check_ptr(alpha));
   CQ_TRY(check_ptr(scale));
-  if (cq::quantize_workspace_bytes(B * H, n) > cq::quantize_static_scratch_bytes())
-    return CQ_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   if (cq::quantize_static_scratch(&scratch) != cudaSuccess) return CQ_ERR_CUDA;
   return cuda_status(cq::launch_quantize(x, dt, B * H, n, bits, layout, codes, alpha, scale,
@@ -319,6 +324,16 @@ cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, con
                          int Hq, int Hkv, int n, int d, int bits, float softmax_scale,
                          cq_calib calib, void* out, void* workspace, size_t ws_bytes,
                          cq_stream_t stream) {
+  return cq_decode_attn_ex(q, dt, k_codes, k_alpha, k_scale, k_layout, v_codes, v_alpha, v_scale, v_layout, B, Hq,
+                           Hkv, n, d, bits, softmax_scale, calib, out, workspace, ws_bytes, nullptr, 0u, stream);
+}
+
+cq_status cq_decode_attn_ex(const void* q, cq_dtype dt, const uint8_t* k_codes, const void* k_alpha,
+                            const void* k_scale, cq_layout k_layout, const uint8_t* v_codes,
+                            const void* v_alpha, const void* v_scale, cq_layout v_layout, int B,
+                            int Hq, int Hkv, int n, int d, int bits, float softmax_scale,
+                            cq_calib calib, void* out, void* workspace, size_t ws_bytes,
+                            int* status, unsigned wait_probes, cq_stream_t stream) {
   if (!valid_dtype(dt)) return CQ_ERR_INVALID_ARG;
   CQ_TRY(check_shape(B, Hq, n, d, bits));
   if (Hkv < 1 || Hq % Hkv) return CQ_ERR_INVALID_ARG;
@@ -337,8 +352,11 @@ cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, con
     return CQ_ERR_UNSUPPORTED;
   const void* ptrs[] = {q, k_codes, k_alpha, k_scale, v_codes, v_alpha, v_scale, out};
   for (const void* p : ptrs) CQ_TRY(check_ptr(p));
+  if (status != nullptr) CQ_TRY(check_ptr(status));
   cq::DecodeArgs a = make_args(q, k_codes, k_alpha, k_scale, v_codes, v_alpha, v_scale, B, Hq, Hkv, n, d, bits,
                                softmax_scale, calib, out);
+  a.status = status;
+  a.wait_probes = wait_probes;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (generic) {
     const size_t need = cq::decode_generic_workspace_bytes(B, Hq, n);

@@ -10,6 +10,14 @@
 
 namespace cq {
 
+// Function attributes (dynamic shared memory, cluster sizes) belong to a device
+// context, so the launchers record per device that they have set them.
+constexpr int kMaxDevices = 64;
+inline int current_device() {
+  int dev = 0;
+  return cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices ? dev : -1;
+}
+
 // ---------------------------------------------------------------- dtypes ----
 template <typename T>
 struct DT;

@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
 
   // ---- 2. post-scaled K weights w_h = sigma q_h (.) s_K in 22-bit fixed point
   const T* sRows = reinterpret_cast<const T*>(F.stage);  // q[4][kD], alpha_K, s_K, alpha_V, s_V
-  wait_copies(&F.bar_rows, 0, err);
+  wait_copies(&F.bar_rows, 0, err, a.wait_probes);
   float w[kG];
   // Every warp runs this (warps 4..7 repeat channels 0..127 and store nothing):
   // a shuffle the compiler cannot prove convergent, e.g. under a branch on the
@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
   // per unit 16 octets x 128 channels
   float mn = FLT_MAX, mx = -FLT_MAX;  // logit range of head tq over this lane's tokens
   for (int u = warp; u < nunits; u += kWarps) {
-    wait_copies(&F.bar_k[u / kWarps], 0, err);
+    wait_copies(&F.bar_k[u / kWarps], 0, err, a.wait_probes);
     uint32_t af[4][4];  // A fragments of chunks c = 0..3 (rows = octets 16u + {g, g+8})
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
     if (grp == 0) F.lsum[warp][h] = lsum;
   }
-  wait_copies(&F.bar_v, 0, err);
+  wait_copies(&F.bar_v, 0, err, a.wait_probes);
   __syncthreads();  // the weight fragments are complete
 
   // ---- 6. V side: warp pair p = warp / 2 takes tiles p, p + 4, ...; warp parity
@@ -457,6 +457,7 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
     }
   }
   if (*err && t == 0) {  // let copies still in flight land before the CTA's memory is reused
+    report_timeout(a.status);
     tc::mbar_wait(&F.bar_rows, 0, kSpin);
     tc::mbar_wait(&F.bar_v, 0, kSpin);
     for (int i = 0; i < nkbox; ++i) tc::mbar_wait(&F.bar_k[i], 0, kSpin);
@@ -466,7 +467,10 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
 template <typename T, int S>
 cudaError_t run_slice(const DecodeArgs& a, int rows, int cl, cudaStream_t stream) {
   const size_t smem = smem_bytes(S) + 1024;  // slack to align the codes to the 1024-byte swizzle atom
-  static bool attr_set = false;  // benign race: every caller sets the same value
+  static bool attr_sets[kMaxDevices];  // per device (benign race: every caller sets the same value)
+  const int attr_dev = current_device();
+  if (attr_dev < 0) return cudaErrorInvalidDevice;
+  bool& attr_set = attr_sets[attr_dev];
   if (!attr_set) {
     const cudaError_t e =
         cudaFuncSetAttribute(k_decode_mma<T, S>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

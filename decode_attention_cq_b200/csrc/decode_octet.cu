@@ -414,6 +414,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     float l = 0.f;
     for (int q = 0; q < 4; ++q) l += S.red[q][t][0];
     S.part_l[t] = failed ? __int_as_float(0x7fc00000) : l;
+    if (failed && t == 0 && a.status != nullptr) atomicOr(a.status, CQ_DEVICE_WAIT_TIMEOUT);
   }
   tc::cluster_sync();
 
@@ -463,13 +464,14 @@ int pick_cluster(int rows, int nk, int sms) {
 
 template <typename T>
 cudaError_t run(const DecodeArgs& a, cudaStream_t stream) {
-  static int sms = 0;  // SM count of device 0 class parts; only sizes the cluster choice
-  if (sms == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      sms = 148;
+  static int sm_counts[kMaxDevices];  // per device; only sizes the cluster choice
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  if (sm_counts[dev] == 0) {
+    int c = 0;
+    sm_counts[dev] = cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? c : 148;
   }
+  const int sms = sm_counts[dev];
   const int rows = a.B * a.Hkv;
   const int nk = (a.n + kKTile - 1) / kKTile;
   const int cl = pick_cluster(rows, nk, sms);
@@ -477,7 +479,10 @@ cudaError_t run(const DecodeArgs& a, cudaStream_t stream) {
   const int slice_tokens = ((nk + cl - 1) / cl) * kKTile;
   size_t smem = align1k(sizeof(Smem)) + (size_t)kG * slice_tokens * sizeof(float);
   if (smem < kMinSmem) smem = kMinSmem;
-  static bool attr_set = false;  // benign race: every caller sets the same value
+  static bool attr_sets[kMaxDevices];  // per device (benign race: every caller sets the same value)
+  const int attr_dev = current_device();
+  if (attr_dev < 0) return cudaErrorInvalidDevice;
+  bool& attr_set = attr_sets[attr_dev];
   if (!attr_set) {
     const size_t max_smem = align1k(sizeof(Smem)) + (size_t)kG * kMaxSlice * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(k_decode_octet<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,

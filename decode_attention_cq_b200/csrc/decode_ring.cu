@@ -495,6 +495,7 @@ __global__ void __launch_bounds__(kThreads, ring_slots<BITS>() == 2 ? 3 : 2)
     }
   }
   if (*err && t == 0) {  // let copies still in flight land before the CTA's memory is reused
+    report_timeout(a.status);
     tc::mbar_wait(&F.bar_rows, 0, kSpin);
     for (int gi = nchunks - kSlots; gi < nchunks; ++gi)
       if (gi >= 0) tc::mbar_wait(&F.full[gi % kSlots], (uint32_t)(gi / kSlots) & 1u, kSpin);
@@ -510,7 +511,10 @@ cudaError_t run_bits(const DecodeArgs& a, cudaStream_t stream) {
   const int cl = (nvt + per - 1) / per;
   if (cl > kMaxCl || (long long)rows * cl > 0x7fffffffLL) return cudaErrorNotSupported;
   const size_t smem = ring_smem_bytes<T, BITS>() + 1024;  // slack to align to the 1024-byte swizzle atom
-  static bool attr_set = false;  // benign race: every caller sets the same values
+  static bool attr_sets[kMaxDevices];  // per device (benign race: every caller sets the same value)
+  const int attr_dev = current_device();
+  if (attr_dev < 0) return cudaErrorInvalidDevice;
+  bool& attr_set = attr_sets[attr_dev];
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(k_decode_ring<T, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);

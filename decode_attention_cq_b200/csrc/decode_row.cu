@@ -713,6 +713,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc::tmem_dealloc(tmem, tmem_cols);
   }
   if (t == 0 && *err) {
+    report_timeout(a.status);
     for (int s = 0; s < kSlots; ++s)
       if (F.uses[s] > 0) tc::mbar_wait(&F.full[s], (F.uses[s] - 1) & 1u, kSpin);
   }
@@ -728,7 +729,10 @@ uint32_t tmem_cols_for(int tiles) {
 
 template <typename T, bool kSplit>
 cudaError_t set_row_attributes(size_t smem) {
-  static bool attr_set = false;  // benign race: every caller sets the same value
+  static bool attr_sets[kMaxDevices];  // per device (benign race: every caller sets the same value)
+  const int attr_dev = current_device();
+  if (attr_dev < 0) return cudaErrorInvalidDevice;
+  bool& attr_set = attr_sets[attr_dev];
   if (attr_set) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(k_decode_row<T, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess)  // two CTAs per SM need the largest shared-memory carve-out

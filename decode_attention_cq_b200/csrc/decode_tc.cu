@@ -538,37 +538,32 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
   }
 
+  if (t == 0 && *err) report_timeout(a.status);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
-int device_sms() {
-  static int sms[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (sms[dev] == 0) {
-    int c = 0;
-    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    sms[dev] = c;
-  }
-  return sms[dev];
-}
-
 template <typename T>
 cudaError_t run(const DecodeArgs& a, cudaStream_t stream) {
   const int rows = a.B * a.Hkv;
-  const int sms = device_sms();
-  if (sms <= 0) return cudaErrorNoDevice;
-  // function attributes apply per device context: set them on every launch (a cheap host call)
-  cudaError_t e = cudaFuncSetAttribute(k_decode_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemTc);
-  if (e != cudaSuccess) return e;
+  static int sms[kMaxDevices];  // per device: SM count, 0 until the attributes are set
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  if (sms[dev] == 0) {
+    int c = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_decode_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemTc);
+    if (e != cudaSuccess) return e;
+    sms[dev] = c;
+  }
   CUtensorMap kmap;
   if (!encode_3d(&kmap, a.k_codes, kD, (uint64_t)(a.n + 7) / 8, (uint64_t)rows, kBlkOct,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  const int grid = rows < sms ? rows : sms;
+  const int grid = rows < sms[dev] ? rows : sms[dev];
   k_decode_tc<T><<<grid, kThreadsTc, kSmemTc, stream>>>(a, rows, kmap);
   return cudaGetLastError();
 }

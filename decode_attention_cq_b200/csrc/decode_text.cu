@@ -230,7 +230,10 @@ cudaError_t launch_text_merge(const DecodeArgs& a, cq_dtype dt, const void* k_te
   const int rows = a.B * a.Hkv;
   if (dt == CQ_F16 && n_text > 0) {
     constexpr size_t kSmem = (size_t)kSlots * txt::kChunkBytes + 1024;  // ring + alignment
-    static bool attr_set = false;  // benign race: every caller sets the same value
+    static bool attr_sets[kMaxDevices];  // per device (benign race: every caller sets the same value)
+    const int attr_dev = current_device();
+    if (attr_dev < 0) return cudaErrorInvalidDevice;
+    bool& attr_set = attr_sets[attr_dev];
     if (!attr_set) {
       const cudaError_t e =
           cudaFuncSetAttribute(k_text_merge_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);

@@ -14,6 +14,9 @@ constexpr int kD = 128;  // head dimension supported by every kernel
 // ---- quantize.cu
 int quantize_splits(int rows, int n);
 size_t quantize_workspace_bytes(int rows, int n);
+// Whether cq_quantize_kv takes the two-launch path that keeps per-split
+// statistics in the workspace (the single-read fill uses none).
+bool quantize_uses_workspace(int rows, int n);
 cudaError_t launch_quantize(const void* x, cq_dtype dt, int rows, int n, int bits, cq_layout layout,
                             uint8_t* codes, void* alpha, void* scale, void* workspace,
                             cudaStream_t stream);
@@ -51,6 +54,12 @@ struct DecodeArgs {
   const void* k_text = nullptr;
   const void* v_text = nullptr;
   int n_text = 0;
+  // Device status word (may be null): a CTA whose bounded wait ran out ORs
+  // CQ_DEVICE_WAIT_TIMEOUT into it (its rows are NaN).
+  int* status = nullptr;
+  // Probes of each wait for a copy in k_decode_mma (whose copies are issued once
+  // per launch) before it gives up; 0 = the default bound (about a second).
+  uint32_t wait_probes = 0;
 };
 size_t decode_generic_workspace_bytes(int B, int Hq, int n);
 cudaError_t launch_decode_generic(const DecodeArgs& a, cq_dtype dt, void* workspace,

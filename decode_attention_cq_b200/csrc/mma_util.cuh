@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "calibq.h"
 #include "tc.cuh"
 
 namespace cq {
@@ -96,9 +97,22 @@ __device__ __forceinline__ int logit_pos(int unit, int k, int h, int o) {
 }
 
 // Every thread waits for the copy phase; a wait that runs out flags the CTA
-// (its outputs become NaN) instead of hanging.
-__device__ __forceinline__ void wait_copies(uint64_t* bar, uint32_t parity, volatile int* err) {
-  if (!tc::mbar_wait(bar, parity, kSpin)) *err = 1;
+// (its outputs become NaN) instead of hanging. probes = 0: the default bound
+// (try_wait, about a second); otherwise that many non-suspending probes.
+__device__ __forceinline__ void wait_copies(uint64_t* bar, uint32_t parity, volatile int* err,
+                                            uint32_t probes = 0) {
+  bool ok = false;
+  if (probes == 0) {
+    ok = tc::mbar_wait(bar, parity, kSpin);
+  } else {
+    for (uint32_t i = 0; i < probes && !ok; ++i) ok = tc::mbar_test_wait(bar, parity);
+  }
+  if (!ok) *err = 1;
+}
+
+// Report a CTA's timed-out wait in the caller's status word (one thread).
+__device__ __forceinline__ void report_timeout(int* status) {
+  if (status != nullptr) atomicOr(status, CQ_DEVICE_WAIT_TIMEOUT);
 }
 
 // The same for a whole warp: every lane probes without suspending and the warp

@@ -430,14 +430,17 @@ cudaError_t launch_fill(const T* x, int rows, int n, uint8_t* codes, T* alpha, T
   // pad brings static + dynamic to 46 KB: more than 228 KB / 5, and within the
   // 48 KB a launch may use without opting in.
   constexpr int kTotal = 46 * 1024;
-  static int pad = -1;  // benign race: every caller computes the same values
-  if (pad < 0) {
+  static int pads[kMaxDevices];  // per device, + 1 once set (benign race: every caller computes the same values)
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  if (pads[dev] == 0) {
     cudaError_t e = cudaFuncSetAttribute(k_fill<T, BITS, LAYOUT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     cudaFuncAttributes fa;
     if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, k_fill<T, BITS, LAYOUT>);
     if (e != cudaSuccess) return e;
-    pad = fa.sharedSizeBytes < (size_t)kTotal ? kTotal - (int)fa.sharedSizeBytes : 0;
+    pads[dev] = 1 + (fa.sharedSizeBytes < (size_t)kTotal ? kTotal - (int)fa.sharedSizeBytes : 0);
   }
+  const int pad = pads[dev] - 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(rows * cl), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -475,11 +478,16 @@ int quantize_splits(int rows, int n) {
   return s < 1 ? 1 : s;
 }
 
+bool quantize_uses_workspace(int rows, int n) {
+  return !(fill_tile_tokens(n) > 0 &&
+           (long long)rows * ((n + fill_tile_tokens(n) - 1) / fill_tile_tokens(n)) <= 0x7fffffffLL);
+}
+
 template <typename T>
 static cudaError_t launch_quantize_t(const T* x, int rows, int n, int bits, cq_layout layout,
                                      uint8_t* codes, T* alpha, T* scale, float* part,
                                      cudaStream_t stream) {
-  if (fill_tile_tokens(n) > 0 && (long long)rows * ((n + fill_tile_tokens(n) - 1) / fill_tile_tokens(n)) <= 0x7fffffffLL) {
+  if (!quantize_uses_workspace(rows, n)) {
     cudaError_t e;
     if (layout == CQ_LAYOUT_CANONICAL)
       e = launch_fill_bits<T, CQ_LAYOUT_CANONICAL>(x, rows, n, bits, codes, alpha, scale, stream);
@@ -544,7 +552,9 @@ size_t quantize_workspace_bytes(int rows, int n) {
 // partials live in a file-scope device array instead of a caller workspace.
 // Every GPU that loads the library holds it until the process exits. Host
 // code must not hand the symbol itself to a kernel (it is a host-side stand-in
-// for the device array), so its device address is looked up once per device.
+// for the device array), so its device address is looked up once per device
+// (with that device current) and kept; cudaDeviceReset makes that address
+// stale, so no call may follow a reset of a device this process used.
 #include <mutex>
 
 namespace cq {
@@ -553,7 +563,6 @@ namespace {
 constexpr size_t kStaticScratchBytes = 4u << 20;  // 4 MiB = 4096 (row, split) partials
 static __device__ __align__(256) unsigned char g_quantize_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 256;
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 }  // namespace

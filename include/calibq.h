@@ -158,15 +158,19 @@ cq_status cq_quantize_kv(const void* x, cq_dtype dt, int B, int H, int n, int d,
  * synchronize the device. This entry point takes the same arguments as
  * cq_quantize_kv minus the workspace, allocates nothing (no cudaMalloc, no
  * cudaFree, no allocating library routine) and keeps its scratch -- the
- * per-split channel minima and maxima -- in a fixed 4 MiB array compiled into
- * the library, which every GPU that loads the library holds until the
- * process exits.
+ * per-split channel minima and maxima of the two-launch path that rows with
+ * n > 16384 take -- in a fixed 4 MiB array compiled into the library, which
+ * every GPU that loads the library holds until the process exits. Rows with
+ * n <= 16384 take the single-read fill, which needs no scratch at all.
  *
- *  - Limit: requests whose scratch (cq_quantize_kv_workspace_size) exceeds
- *    4 MiB return CQ_ERR_UNSUPPORTED and launch nothing.
+ *  - Limit: a request on the two-launch path whose scratch
+ *    (cq_quantize_kv_workspace_size) exceeds 4 MiB returns
+ *    CQ_ERR_UNSUPPORTED and launches nothing; this is decided from the sizes
+ *    alone, before the pointers are looked at.
  *  - The first call on each device looks up that device's address of the
- *    array (with the device current); make that first call before any stream
- *    capture.
+ *    array (with the device current) and keeps it; make that first call
+ *    before any stream capture. cudaDeviceReset invalidates the kept address:
+ *    do not call this entry point on a device after resetting it.
  *  - Every call, on any stream, shares the one array: calls whose kernels
  *    overlap on the GPU race with each other. Serialize them (one stream, or
  *    events). The array keeps the previous call's contents; nothing in it has
@@ -214,6 +218,42 @@ cq_status cq_decode_attn(const void* q, cq_dtype dt, const uint8_t* k_codes, con
                          int Hq, int Hkv, int n, int d, int bits, float softmax_scale,
                          cq_calib calib, void* out, void* workspace, size_t ws_bytes,
                          cq_stream_t stream);
+
+/* Bit of the device status word of cq_decode_attn_ex: a bounded wait of a
+ * decode kernel ran out; the rows of the CTAs concerned were written as NaN. */
+#define CQ_DEVICE_WAIT_TIMEOUT 1
+
+/*
+ * cq_decode_attn with a device-side error report. Every wait of the decode
+ * kernels for data (copies from global memory, tensor-core results) is
+ * bounded; a wait that runs out does not hang the GPU: the CTA writes NaN to
+ * its output rows, lets the copies it issued land, and returns. The host-side
+ * status (the return value) cannot know about it, since the call returns
+ * before the kernels run; this entry point reports it on the device instead:
+ *
+ *   status       NULL, or device memory holding one int (16-byte aligned, like
+ *                every pointer of this library): when any CTA's wait ran out,
+ *                CQ_DEVICE_WAIT_TIMEOUT is ORed into it. Nothing else is
+ *                written there; the caller zeroes it before the call and reads
+ *                it after synchronizing `stream`.
+ *   wait_probes  0 for the kernels' own bounds (about a second of waiting).
+ *                Otherwise each wait for a copy in "k_decode_mma" (the kernel
+ *                whose copies are all issued at the start of the launch) gives
+ *                up after that many non-blocking probes: a diagnostic that
+ *                exercises the timeout path (1 makes it give up while the
+ *                copies are still in flight). The other kernels keep their own
+ *                bounds, since their copy rings must not be re-armed before a
+ *                copy has landed.
+ *
+ * Everything else is as for cq_decode_attn, which is this call with
+ * status = NULL and wait_probes = 0.
+ */
+cq_status cq_decode_attn_ex(const void* q, cq_dtype dt, const uint8_t* k_codes, const void* k_alpha,
+                            const void* k_scale, cq_layout k_layout, const uint8_t* v_codes,
+                            const void* v_alpha, const void* v_scale, cq_layout v_layout, int B,
+                            int Hq, int Hkv, int n, int d, int bits, float softmax_scale,
+                            cq_calib calib, void* out, void* workspace, size_t ws_bytes,
+                            int* status, unsigned wait_probes, cq_stream_t stream);
 
 /*
  * Name of the kernel that cq_decode_attn launches for these layouts and sizes

@@ -165,3 +165,13 @@ def test_host_pointer_is_rejected(lib):
     addr = (ctypes.addressof(buf) + 15) & ~15
     st = lib.cq_dequant(addr, addr, addr, 0, 0, 1, 1, 4, 128, 1, addr, None)
     assert st in (cq.CQ_ERR_INVALID_ARG, cq.CQ_ERR_CUDA)
+
+
+def test_noalloc_refuses_oversized_scratch_before_pointers(lib):
+    """cq_quantize_kv_noalloc decides its scratch limit from the sizes alone:
+    only the two-launch path (n > 16384) uses the fixed 4 MiB array."""
+    C = cq.LAYOUT_CANONICAL
+    f = lib.cq_quantize_kv_noalloc
+    assert f(None, 0, 1, 4097, 16385, 128, 1, C, None, None, None, None) == cq.CQ_ERR_UNSUPPORTED
+    assert f(None, 0, 1, 4096, 16385, 128, 1, C, None, None, None, None) == cq.CQ_ERR_INVALID_ARG
+    assert f(None, 0, 1, 4097, 1, 128, 1, C, None, None, None, None) == cq.CQ_ERR_INVALID_ARG  # fill path: no limit

@@ -29,3 +29,26 @@ def test_figure_reproduces_the_calibration_effect(cuda_device):
     assert s["Exact"]["kl"] == pytest.approx(0.0, abs=1e-12)
     for r in s.values():
         assert sum(r["hist"]) == pytest.approx(32 * 1200)
+
+
+@pytest.mark.gpu
+def test_figure_series_match_the_oracle(cuda_device):
+    """The three series element by element against the oracle on the same
+    seeded inputs: Exact = sigma q.k, Quant = the same on the oracle's 1-bit
+    dequantized keys (rounded once to f16, as the library stores them),
+    Quant-C = the oracle's calibration map g of Quant."""
+    from decode_attention_cq_b200 import synth
+
+    n, tau, seed = 1200, (0.8, 0.9), 3
+    series = score_figure.score_series(n=n, tau=tau, seed=seed, device=cuda_device)
+    q, k, _ = synth.make_case(1, 32, 8, n, 128, "f16", outliers=4, seed=seed, device=cuda_device)  # as the tool draws them
+    qd, kd = q.cpu().double().numpy(), k.cpu().double().numpy()
+    kq = oracle.quantize_cache(kd, 1, "f16")
+    k_hat = oracle.dequantize(kq["codes"], kq["alpha"], kq["scale"]).astype(np.float16).astype(np.float64)
+    want = {"Exact": oracle.scores_dequantized(qd, kd)[0],
+            "Quant": oracle.scores_dequantized(qd, k_hat)[0]}
+    want["Quant-C"] = oracle.calibrate(want["Quant"], *tau)
+    for name, ref in want.items():
+        got = series[name].cpu().numpy()
+        assert got.shape == ref.shape
+        assert np.allclose(got, ref, rtol=1e-9, atol=1e-9 * np.abs(ref).max()), name
