@@ -220,6 +220,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const Ring R{&kmap, &vmap, &ktmap, &vtmap, row, tile0, nchunk, 2 * nchunk + 2 * ntp};
   volatile int* err = &F.err;
   if constexpr (kSplit) tc::cluster_arrive_relaxed();  // matched by the wait before the first peer store
+  // a launch of split rows that follows this one on the stream may start now
+  if constexpr (!kSplit) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---- 1. barriers, tensor memory, the query and statistics rows, the first
   // chunks: warp 1 sets up and issues the copies while warp 0 allocates
@@ -742,36 +744,6 @@ cudaError_t set_row_attributes(size_t smem) {
   return e;
 }
 
-// The stream and events a launch with split rows forks onto, one set per host
-// thread and device (captured into a CUDA graph like the caller's stream).
-struct SideStream {
-  int dev = -1;
-  cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
-};
-
-cudaError_t side_stream(SideStream*& out) {
-  thread_local SideStream side;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (side.dev != dev) {
-    if (side.s != nullptr) {  // another device: the old handles belong to it
-      cudaStreamDestroy(side.s);
-      cudaEventDestroy(side.fork);
-      cudaEventDestroy(side.join);
-      side = SideStream{};
-    }
-    if ((e = cudaStreamCreateWithFlags(&side.s, cudaStreamNonBlocking)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&side.fork, cudaEventDisableTiming)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&side.join, cudaEventDisableTiming)) != cudaSuccess)
-      return e;
-    side.dev = dev;
-  }
-  out = &side;
-  return cudaSuccess;
-}
-
 int device_sms() {
   static int count[64] = {};  // per device ordinal; 0 until read
   int dev = 0, c = 0;
@@ -804,34 +776,33 @@ cudaError_t run_row(const DecodeArgs& a, cudaStream_t stream) {
 
   const int split = decode_row_split_rows(rows, a.n, a.n_text == 0 && a.part_o == nullptr);
   const int whole = rows - split;
-  SideStream* side = nullptr;
-  if (split > 0) {
-    if ((e = set_row_attributes<T, true>(smem)) != cudaSuccess || (e = side_stream(side)) != cudaSuccess) return e;
-    if ((e = cudaEventRecord(side->fork, stream)) != cudaSuccess ||
-        (e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess)
-      return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(2 * split), 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = side->s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if ((e = cudaLaunchKernelEx(&cfg, k_decode_row<T, true>, a, tmem_cols_for((nt + 1) / 2), whole, kmap, vmap,
-                                ktmap, vtmap)) != cudaSuccess ||
-        (e = cudaEventRecord(side->join, side->s)) != cudaSuccess)
-      return e;
-  }
   if (whole > 0) {
     k_decode_row<T, false><<<whole, kThreads, smem, stream>>>(a, tmem_cols_for(nt), 0, kmap, vmap, ktmap, vtmap);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  if (split > 0) return cudaStreamWaitEvent(stream, side->join, 0);
+  if (split > 0) {
+    // the halves go into the same stream as a programmatic dependent launch:
+    // every whole-row CTA lets it start as soon as it runs, and it reads and
+    // writes nothing of theirs, so its CTAs take SM slots as whole rows finish
+    if ((e = set_row_attributes<T, true>(smem)) != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * split), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if ((e = cudaLaunchKernelEx(&cfg, k_decode_row<T, true>, a, tmem_cols_for((nt + 1) / 2), whole, kmap, vmap,
+                                ktmap, vtmap)) != cudaSuccess)
+      return e;
+  }
   return cudaSuccess;
 }
 
@@ -842,7 +813,8 @@ bool decode_row_supports(int n) { return n >= 1 && n <= kMaxTiles * kTile; }
 // Two rows per SM run at once. Past two full waves, the rows beyond a whole
 // number of SM counts would leave some SMs one row more than the others; in
 // a plain decode those rows run as halves on 2-CTA clusters, in a second
-// launch on a side stream, so that the halves spread over the SMs. Only while
+// launch (programmatic dependent: it overlaps the whole rows on the same
+// stream), so that the halves spread over the SMs. Only while
 // they are at most half the SM count: beyond that most SMs would take a half
 // on top of their whole rows and the halves' own cost (set-up, the two
 // exchanges) outweighs the balance (measured on B200: 512 rows of 8192 tokens

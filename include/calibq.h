@@ -289,11 +289,10 @@ const char* cq_decode_kernel_name(cq_layout k_layout, cq_layout v_layout, int B,
  *   them, and that a plain 1-bit call on the row kernel with more than two
  *   waves of rows (two rows per SM) runs the rows beyond a whole number of SM
  *   counts, when they are at most half the SM count, as half rows on 2-CTA
- *   clusters, in a second launch on a side stream forked from and joined back
- *   into `stream`. That side stream and its two events are created once per
- *   host thread and device, by the first such call; make that call outside
- *   stream capture (a warm-up call before capturing a CUDA graph), since a
- *   capture in the global mode does not allow creating them.
+ *   clusters in a second launch on the same stream (a programmatic dependent
+ *   launch: it overlaps the whole rows, and reads or writes nothing of theirs).
+ *   No call creates streams or events; every call can be captured into a
+ *   CUDA graph, the first one of a process included.
  */
 int cq_decode_launch_count(cq_layout k_layout, cq_layout v_layout, int B, int Hq, int Hkv, int n, int d, int bits,
                            int n_text);
