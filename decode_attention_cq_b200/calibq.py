@@ -245,7 +245,7 @@ def cq_decode_attn(q: torch.Tensor, k: QuantizedCache, v: QuantizedCache, *,
     _, Hkv, n, _ = k.shape
     if out is None:
         out = torch.empty_like(q)
-    if workspace is None:
+    if workspace is None and k.layout == LAYOUT_CANONICAL:  # the octet path takes none
         ws = cq_decode_attn_workspace_size(k.layout, v.layout, B, Hq, Hkv, n, d, k.bits)
         workspace = torch.empty(ws, dtype=torch.uint8, device=q.device) if ws else None
     cal = _calib(bool(calib[0]), float(calib[1]), float(calib[2]))
@@ -271,7 +271,7 @@ def cq_decode_attn_ex(q: torch.Tensor, k: QuantizedCache, v: QuantizedCache, sta
     _, Hkv, n, _ = k.shape
     if out is None:
         out = torch.empty_like(q)
-    if workspace is None:
+    if workspace is None and k.layout == LAYOUT_CANONICAL:  # the octet path takes none
         ws = cq_decode_attn_workspace_size(k.layout, v.layout, B, Hq, Hkv, n, d, k.bits)
         workspace = torch.empty(ws, dtype=torch.uint8, device=q.device) if ws else None
     if status.dtype != torch.int32 or not status.is_cuda:

@@ -6,6 +6,8 @@
 
 #include <limits>
 
+#include <cuda.h>  // CUdeviceptr, CUresult (the driver entry point, no libcuda link)
+
 #include "calibq.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -23,9 +25,43 @@ bool valid_layout(cq_layout l) {
 }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// cuMemGetAddressRange through the runtime's driver entry point (the library
+// does not link libcuda): the extent of the allocation that holds a pointer.
+using GetAddressRange = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
+GetAddressRange address_range_fn() {
+  static const GetAddressRange fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<GetAddressRange>(p);
+  }();
+  return fn;
+}
+
+// Allocations that passed check_ptr on this host thread: [base, end) of device
+// memory of device `dev`, or of managed memory (dev = -1). A call passes up to
+// ten pointers, most of them into the same few allocations, and a decode loop
+// passes the same buffers every step; a pointer inside a remembered allocation
+// is accepted without a driver query (each costs a few tenths of a
+// microsecond). Replaced round robin.
+struct SeenAlloc {
+  uintptr_t base = 0, end = 0;
+  int dev = -2;
+};
+constexpr int kSeenAllocs = 16;
+thread_local SeenAlloc g_seen[kSeenAllocs];
+thread_local int g_seen_next = 0;
+
 // Device memory of the current device (or managed memory) and 16-byte aligned.
 cq_status check_ptr(const void* p) {
   if (p == nullptr || !aligned16(p)) return CQ_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CQ_ERR_CUDA;
+  const uintptr_t u = reinterpret_cast<uintptr_t>(p);
+  for (const SeenAlloc& a : g_seen)
+    if (u >= a.base && u < a.end && (a.dev == dev || a.dev == -1)) return CQ_OK;
   cudaPointerAttributes attr;
   cudaError_t e = cudaPointerGetAttributes(&attr, p);
   if (e != cudaSuccess) {
@@ -34,9 +70,15 @@ cq_status check_ptr(const void* p) {
   }
   if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
     return CQ_ERR_INVALID_ARG;
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return CQ_ERR_CUDA;
   if (attr.type == cudaMemoryTypeDevice && attr.device != dev) return CQ_ERR_INVALID_ARG;
+  CUdeviceptr base = 0;
+  size_t bytes = 0;
+  const GetAddressRange range = address_range_fn();
+  if (range != nullptr && range(&base, &bytes, (CUdeviceptr)u) == CUDA_SUCCESS && bytes > 0) {
+    g_seen[g_seen_next] = SeenAlloc{(uintptr_t)base, (uintptr_t)base + bytes,
+                                    attr.type == cudaMemoryTypeManaged ? -1 : dev};
+    g_seen_next = (g_seen_next + 1) % kSeenAllocs;
+  }
   return CQ_OK;
 }
 

@@ -11,12 +11,13 @@
  *
  *  - All tensor pointers are DEVICE pointers owned by the caller (device or
  *    managed memory of the current device; host pointers are rejected with
- *    CQ_ERR_INVALID_ARG). The library never allocates device memory in these
- *    calls. Host-side state: the kernel choice set by cq_set_decode_kernel
- *    (process-wide), a small cache of encoded tensor maps per host thread,
- *    and per host thread and device one stream and two events, created by the
- *    first decode that splits rows (cq_decode_launch_count). Calls are
- *    thread-safe.
+ *    CQ_ERR_INVALID_ARG). The library never allocates device memory and
+ *    creates no streams or events in these calls. Host-side state: the kernel
+ *    choice set by cq_set_decode_kernel (process-wide), and per host thread a
+ *    small cache of encoded tensor maps and of the device allocations that
+ *    earlier calls validated (a pointer inside one of those is accepted
+ *    without asking the driver again, so a pointer into memory freed since is
+ *    not caught: pass no dangling pointers). Calls are thread-safe.
  *  - Work is enqueued asynchronously on `stream` (NULL = the legacy default
  *    stream). A returned CQ_OK means the launch was enqueued; kernel faults
  *    surface on the stream like any CUDA error.
@@ -209,6 +210,11 @@ cq_status cq_decode_attn_workspace_size(cq_layout k_layout, cq_layout v_layout, 
  * (OCTET_K, OCTET_V) for d = 128, Hq = 4*Hkv and n <= 65536 at bits = 1
  * (n <= 32768 at bits 2, 4, 8) -- the tensor-core path, one launch per call
  * (two for some batches of the 1-bit row kernel: cq_decode_launch_count).
+ * The octet kernels hold the four query heads of a kv-head in the rows of
+ * one tensor-core tile, so any other ratio Hq/Hkv with the octet layouts
+ * returns CQ_ERR_UNSUPPORTED; such models store their cache in the CANONICAL
+ * layout, whose CUDA-core kernels take any ratio but run several times
+ * slower (about 7x at 1 bit, n = 8192, batch 16 on B200).
  * cq_decode_kernel_name says which kernel a call launches; the 1-bit kernels
  * agree with each other within the output tolerance, not bit for bit.
  */

@@ -79,3 +79,31 @@ def test_octet_path_length_limit(cuda_device):
     with pytest.raises(cq.CalibqError) as e:
         cq.cq_decode_attn(q, kq, vq)
     assert e.value.status == cq.CQ_ERR_UNSUPPORTED
+
+
+def test_validated_allocations_are_remembered_per_allocation(cuda_device):
+    """A pointer inside an allocation that an earlier call validated is
+    accepted without a new driver query; pointers the driver would reject are
+    still rejected after device buffers have been remembered."""
+    x, qc = _qc(cuda_device, n=64, H=4)
+    lib = cq.load()
+    s = torch.cuda.current_stream().cuda_stream
+    ws = torch.empty(cq.cq_quantize_kv_workspace_size(1, 2, 64, 128), dtype=torch.uint8, device=cuda_device)
+
+    def call(xp, codes=qc.codes.data_ptr()):
+        return lib.cq_quantize_kv(xp, 0, 1, 2, 64, 128, 1, 0, codes, qc.alpha.data_ptr(), qc.scale.data_ptr(),
+                                  ws.data_ptr(), ws.numel(), s)
+
+    assert call(x.data_ptr()) == cq.CQ_OK
+    # heads 2..3 of the same tensor: same allocation, 16-byte aligned
+    assert call(x.data_ptr() + 2 * 64 * 128 * 2) == cq.CQ_OK
+    host = torch.empty(64 * 128 * 2, dtype=torch.uint8)
+    assert call(host.data_ptr()) == cq.CQ_ERR_INVALID_ARG
+    assert call(x.data_ptr(), codes=host.data_ptr()) == cq.CQ_ERR_INVALID_ARG
+    assert call(x.data_ptr() + 16 + 2) == cq.CQ_ERR_INVALID_ARG  # misaligned, inside a remembered allocation
+    torch.cuda.synchronize()
+    # the same buffers through the binding, many times: outputs stay exact
+    want = cq.cq_quantize_kv(x, 1, cq.LAYOUT_CANONICAL)
+    for _ in range(3):
+        got = cq.cq_quantize_kv(x, 1, cq.LAYOUT_CANONICAL)
+        assert torch.equal(got.codes, want.codes)
