@@ -8,6 +8,8 @@
 //            alpha and the step (once per row) and the packed codes of its tile.
 #include <float.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -20,10 +22,29 @@ constexpr int kThreads = 256;
 constexpr int kTpr = kD / 8;            // threads per token row (8 channels each)
 constexpr int kRpi = kThreads / kTpr;   // token rows per iteration
 
+// Where the pack functions read token rows from (the row in global memory).
+template <typename T>
+struct GlobalRows {
+  const T* __restrict__ row0;  // token 0 of the (batch, head) row
+  __device__ __forceinline__ void load8(int i, int ch, float (&v)[8]) const {
+    cq::load8(row0 + (size_t)i * kD + ch, v);
+  }
+  // the same eight binary16 values as four packed pairs
+  __device__ __forceinline__ void load8h(int i, int ch, uint32_t (&w)[4]) const {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(row0 + (size_t)i * kD + ch));
+    w[0] = u.x;
+    w[1] = u.y;
+    w[2] = u.z;
+    w[3] = u.w;
+  }
+};
+
 // Per-channel min / max of tokens [i0, i1) of one row; thread j < kD gets
 // channel j's pair. 16 threads cover a token row (8 channels each).
+// smn, smx: kRpi x kD floats each of shared scratch.
 template <typename T>
-__device__ __forceinline__ void tile_minmax(const T* __restrict__ xrow, int i0, int i1, float& a, float& b) {
+__device__ __forceinline__ void tile_minmax(const T* __restrict__ xrow, int i0, int i1, float& a, float& b,
+                                            float (*smn)[kD], float (*smx)[kD]) {
   const int cg = threadIdx.x % kTpr, r = threadIdx.x / kTpr;
   float mn[8], mx[8];
 #pragma unroll
@@ -32,17 +53,43 @@ __device__ __forceinline__ void tile_minmax(const T* __restrict__ xrow, int i0, 
     mx[e] = -FLT_MAX;
   }
   const T* base = xrow + cg * 8;
-#pragma unroll 8
-  for (int i = i0 + r; i < i1; i += kRpi) {
-    float v[8];
-    load8(base + (size_t)i * kD, v);
+  if constexpr (std::is_same<T, half>::value) {
+    // binary16 extremes are binary16 values: packed pairs, no conversions
+    __half2 mn2[4], mx2[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      mn[e] = fminf(mn[e], v[e]);
-      mx[e] = fmaxf(mx[e], v[e]);
+    for (int p = 0; p < 4; ++p) {
+      mn2[p] = __half2half2(__ushort_as_half(0x7c00u));  // +inf
+      mx2[p] = __half2half2(__ushort_as_half(0xfc00u));  // -inf
+    }
+#pragma unroll 8
+    for (int i = i0 + r; i < i1; i += kRpi) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(base + (size_t)i * kD));
+      const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        mn2[p] = __hmin2(mn2[p], h[p]);
+        mx2[p] = __hmax2(mx2[p], h[p]);
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      mn[2 * p] = __low2float(mn2[p]);
+      mn[2 * p + 1] = __high2float(mn2[p]);
+      mx[2 * p] = __low2float(mx2[p]);
+      mx[2 * p + 1] = __high2float(mx2[p]);
+    }
+  } else {
+#pragma unroll 8
+    for (int i = i0 + r; i < i1; i += kRpi) {
+      float v[8];
+      load8(base + (size_t)i * kD, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        mn[e] = fminf(mn[e], v[e]);
+        mx[e] = fmaxf(mx[e], v[e]);
+      }
     }
   }
-  __shared__ float smn[kRpi][kD], smx[kRpi][kD];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     smn[r][cg * 8 + e] = mn[e];
@@ -65,8 +112,9 @@ __global__ void __launch_bounds__(kThreads) k_stats(const T* __restrict__ x, int
   const int row = blockIdx.x, s = blockIdx.y;
   const int per = (n + S - 1) / S;
   const int i0 = s * per, i1 = min(n, i0 + per);
+  __shared__ float smn[kRpi][kD], smx[kRpi][kD];
   float a, b;
-  tile_minmax<T>(x + (size_t)row * n * kD, i0, i1, a, b);
+  tile_minmax<T>(x + (size_t)row * n * kD, i0, i1, a, b, smn, smx);
   if (threadIdx.x < kD) {
     float* out = part + ((size_t)row * S + s) * 2 * kD;
     out[threadIdx.x] = a;
@@ -74,11 +122,35 @@ __global__ void __launch_bounds__(kThreads) k_stats(const T* __restrict__ x, int
   }
 }
 
+// A row's folded statistics, shared by the CTA that packs one of its tiles.
+struct RowStats {
+  float alpha[kD], beta[kD];
+  float inv[kD];     // L / (beta - alpha), 0 for a constant channel
+  uint16_t thr[kD];  // binary16 rows: bits of the smallest binary16 above (alpha + beta) / 2
+};
+
+// 1-bit code of a binary16 value x: [x > (alpha + beta) / 2] (the rounding rule
+// with L = 1, see code1). alpha and beta are binary16 values, so their mean mu is
+// exact in double, and x > mu holds exactly when x >= the smallest binary16 above
+// mu: one packed comparison per two values decides the codes.
+__device__ __forceinline__ uint16_t half_above_mid(float a, float b) {
+  const double mu = ((double)a + (double)b) * 0.5;
+  const uint16_t h = __half_as_ushort(__double2half(mu));  // nearest, ties to even
+  if ((double)__half2float(__ushort_as_half(h)) > mu) return h;  // nearest is above: nothing between
+  if ((h & 0x7fffu) == 0) return 0x0001u;                        // +-0: the smallest subnormal
+  return (h & 0x8000u) ? (uint16_t)(h - 1u) : (uint16_t)(h + 1u);  // one step up
+}
+
+// Per pair of channels (2p, 2p + 1): 0xffff in each half whose value is >= its threshold.
+__device__ __forceinline__ uint32_t ge_mask(uint32_t x2, uint32_t thr2) {
+  return __hge2_mask(*reinterpret_cast<const __half2*>(&x2), *reinterpret_cast<const __half2*>(&thr2));
+}
+
 // Folds the S partials of `row` ([S][min, max][kD], global or shared memory)
 // into shared alpha/beta/inv; with `write` also stores the row's alpha and step.
 template <typename T>
 __device__ __forceinline__ void fold_stats(const float* p, int S, int L, bool write, int row,
-                                           float* s_alpha, float* s_beta, float* s_inv,
+                                           RowStats& st,
                                            T* __restrict__ alpha_out, T* __restrict__ scale_out) {
   if (threadIdx.x < kD) {
     const int j = threadIdx.x;
@@ -87,9 +159,10 @@ __device__ __forceinline__ void fold_stats(const float* p, int S, int L, bool wr
       a = fminf(a, p[s * 2 * kD + j]);
       b = fmaxf(b, p[s * 2 * kD + kD + j]);
     }
-    s_alpha[j] = a;
-    s_beta[j] = b;
-    s_inv[j] = (b > a) ? (float)L / (b - a) : 0.f;
+    st.alpha[j] = a;
+    st.beta[j] = b;
+    st.inv[j] = (b > a) ? (float)L / (b - a) : 0.f;
+    if constexpr (std::is_same<T, half>::value) st.thr[j] = half_above_mid(a, b);
     if (write) {
       alpha_out[(size_t)row * kD + j] = DT<T>::from_float(a);  // exact: an input value
       const double step = __ddiv_rn(__dsub_rn((double)b, (double)a), (double)L);
@@ -100,40 +173,56 @@ __device__ __forceinline__ void fold_stats(const float* p, int S, int L, bool wr
 }
 
 // Canonical layout: each thread turns 8 channels of one token into 8*BITS bits.
-template <typename T, int BITS>
-__device__ __forceinline__ void k_pack_canonical_tile(const T* __restrict__ x, int n, int row, int tile, int tile_tokens,
-    const float* s_alpha, const float* s_beta, const float* s_inv, uint8_t* __restrict__ codes) {
+template <typename T, int BITS, typename Src>
+__device__ __forceinline__ void k_pack_canonical_tile(const Src& src, int n, int row, int tile, int tile_tokens,
+    const RowStats& st, uint8_t* __restrict__ codes) {
   constexpr int L = (1 << BITS) - 1;
   const int cg = threadIdx.x % kTpr, r = threadIdx.x / kTpr;
-  float af[8], inv[8], hi[8], lo[8];
-  double ad[8], bd[8];
+  if constexpr (BITS == 1 && std::is_same<T, half>::value) {
+    // channel 2p's code from the low half of pair p lands on bit 2p, channel
+    // 2p + 1's from the high half on bit 17 + 2p (folded down to 2p + 1)
+    uint32_t th[4];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    af[e] = s_alpha[cg * 8 + e];
-    inv[e] = s_inv[cg * 8 + e];
-    ad[e] = (double)af[e];
-    bd[e] = (double)s_beta[cg * 8 + e];
-    two_sum(af[e], s_beta[cg * 8 + e], hi[e], lo[e]);  // used for 1-bit codes
-  }
-  const int i0 = tile * tile_tokens, i1 = min(n, i0 + tile_tokens);
-  const T* xr = x + (size_t)row * n * kD + cg * 8;
-  uint8_t* cr = codes + (size_t)row * n * (kD * BITS / 8) + cg * BITS;
-  for (int i = i0 + r; i < i1; i += kRpi) {
-    float v[8];
-    load8(xr + (size_t)i * kD, v);
-    uint64_t packed = 0;
+    for (int p = 0; p < 4; ++p) th[p] = st.thr[cg * 8 + 2 * p] | ((uint32_t)st.thr[cg * 8 + 2 * p + 1] << 16);
+    const int i0 = tile * tile_tokens, i1 = min(n, i0 + tile_tokens);
+    uint8_t* cr = codes + (size_t)row * n * (kD / 8) + cg;
+    for (int i = i0 + r; i < i1; i += kRpi) {
+      uint32_t w[4], acc = 0;
+      src.load8h(i, cg * 8, w);
+#pragma unroll
+      for (int p = 0; p < 4; ++p) acc |= ge_mask(w[p], th[p]) & ((1u << (2 * p)) | (1u << (17 + 2 * p)));
+      cr[(size_t)i * (kD / 8)] = (uint8_t)(acc | (acc >> 16));
+    }
+  } else {
+    float af[8], inv[8], hi[8], lo[8];
+    double ad[8], bd[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      if constexpr (BITS == 1)
-        packed |= (uint64_t)code1(v[e], hi[e], lo[e]) << e;
-      else
-        packed |= (uint64_t)quant_code(v[e], af[e], inv[e], ad[e], bd[e], L) << (e * BITS);
+      af[e] = st.alpha[cg * 8 + e];
+      inv[e] = st.inv[cg * 8 + e];
+      ad[e] = (double)af[e];
+      bd[e] = (double)st.beta[cg * 8 + e];
+      two_sum(af[e], st.beta[cg * 8 + e], hi[e], lo[e]);  // used for 1-bit codes
     }
-    uint8_t* dst = cr + (size_t)i * (kD * BITS / 8);
-    if (BITS == 1) *dst = (uint8_t)packed;
-    if (BITS == 2) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
-    if (BITS == 4) *reinterpret_cast<uint32_t*>(dst) = (uint32_t)packed;
-    if (BITS == 8) *reinterpret_cast<uint64_t*>(dst) = packed;
+    const int i0 = tile * tile_tokens, i1 = min(n, i0 + tile_tokens);
+    uint8_t* cr = codes + (size_t)row * n * (kD * BITS / 8) + cg * BITS;
+    for (int i = i0 + r; i < i1; i += kRpi) {
+      float v[8];
+      src.load8(i, cg * 8, v);
+      uint64_t packed = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if constexpr (BITS == 1)
+          packed |= (uint64_t)code1(v[e], hi[e], lo[e]) << e;
+        else
+          packed |= (uint64_t)quant_code(v[e], af[e], inv[e], ad[e], bd[e], L) << (e * BITS);
+      }
+      uint8_t* dst = cr + (size_t)i * (kD * BITS / 8);
+      if (BITS == 1) *dst = (uint8_t)packed;
+      if (BITS == 2) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
+      if (BITS == 4) *reinterpret_cast<uint32_t*>(dst) = (uint32_t)packed;
+      if (BITS == 8) *reinterpret_cast<uint64_t*>(dst) = packed;
+    }
   }
 }
 
@@ -141,40 +230,64 @@ template <typename T, int BITS>
 __global__ void __launch_bounds__(kThreads) k_pack_canonical(
     const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
     uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
-  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
+  __shared__ RowStats st;
   const int row = blockIdx.x;
-  fold_stats<T>(part + (size_t)row * S * 2 * kD, S, (1 << BITS) - 1, blockIdx.y == 0, row, s_alpha, s_beta, s_inv, alpha_out,
+  fold_stats<T>(part + (size_t)row * S * 2 * kD, S, (1 << BITS) - 1, blockIdx.y == 0, row, st, alpha_out,
                 scale_out);
-  k_pack_canonical_tile<T, BITS>(x, n, row, blockIdx.y, tile_tokens, s_alpha, s_beta, s_inv, codes);
+  k_pack_canonical_tile<T, BITS>(GlobalRows<T>{x + (size_t)row * n * kD}, n, row, blockIdx.y, tile_tokens, st, codes);
 }
 
 // OCTET_K layout (bits = 1): a thread owns one token octet (8 tokens) x 8
 // channels, i.e. 8 consecutive bytes of the layout.
-template <typename T>
-__device__ __forceinline__ void k_pack_octet_k_tile(const T* __restrict__ x, int n, int row, int tile, int tile_tokens,
-    const float* s_alpha, const float* s_beta, const float* s_inv, uint8_t* __restrict__ codes) {
+template <typename T, typename Src>
+__device__ __forceinline__ void k_pack_octet_k_tile(const Src& src, int n, int row, int tile, int tile_tokens,
+    const RowStats& st, uint8_t* __restrict__ codes) {
   const int cb = threadIdx.x % kTpr, r = threadIdx.x / kTpr;
-  float hi[8], lo[8];  // alpha + beta of the thread's channels as an exact pair
+  if constexpr (std::is_same<T, half>::value) {
+    // token k's codes of channel pair p go to bits k (channel 2p) and 16 + k
+    // (channel 2p + 1) of acc[p]; two byte permutes give the 8 channel bytes
+    uint32_t th[4];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) two_sum(s_alpha[cb * 8 + e], s_beta[cb * 8 + e], hi[e], lo[e]);
-  const int octets = (n + 7) / 8;
-  const int m0 = tile * (tile_tokens / 8), m1 = min(octets, m0 + tile_tokens / 8);
-  const T* xr = x + (size_t)row * n * kD + cb * 8;
-  uint8_t* cr = codes + (size_t)row * octets * kD + cb * 8;
-  for (int m = m0 + r; m < m1; m += kRpi) {
-    uint64_t bytes = 0;
+    for (int p = 0; p < 4; ++p) th[p] = st.thr[cb * 8 + 2 * p] | ((uint32_t)st.thr[cb * 8 + 2 * p + 1] << 16);
+    const int octets = (n + 7) / 8;
+    const int m0 = tile * (tile_tokens / 8), m1 = min(octets, m0 + tile_tokens / 8);
+    uint8_t* cr = codes + (size_t)row * octets * kD + cb * 8;
+    for (int m = m0 + r; m < m1; m += kRpi) {
+      uint32_t acc[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int i = 8 * m + k;
-      if (i < n) {
-        float v[8];
-        load8(xr + (size_t)i * kD, v);
+      for (int k = 0; k < 8; ++k) {
+        if (8 * m + k < n) {
+          uint32_t w[4];
+          src.load8h(8 * m + k, cb * 8, w);
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          bytes |= (uint64_t)code1(v[e], hi[e], lo[e]) << (8 * e + k);
+          for (int p = 0; p < 4; ++p) acc[p] |= ge_mask(w[p], th[p]) & (0x00010001u << k);
+        }
       }
+      *reinterpret_cast<uint2*>(cr + (size_t)m * kD) =
+          make_uint2(__byte_perm(acc[0], acc[1], 0x6420), __byte_perm(acc[2], acc[3], 0x6420));
     }
-    *reinterpret_cast<uint64_t*>(cr + (size_t)m * kD) = bytes;
+  } else {
+    float hi[8], lo[8];  // alpha + beta of the thread's channels as an exact pair
+#pragma unroll
+    for (int e = 0; e < 8; ++e) two_sum(st.alpha[cb * 8 + e], st.beta[cb * 8 + e], hi[e], lo[e]);
+    const int octets = (n + 7) / 8;
+    const int m0 = tile * (tile_tokens / 8), m1 = min(octets, m0 + tile_tokens / 8);
+    uint8_t* cr = codes + (size_t)row * octets * kD + cb * 8;
+    for (int m = m0 + r; m < m1; m += kRpi) {
+      uint64_t bytes = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int i = 8 * m + k;
+        if (i < n) {
+          float v[8];
+          src.load8(i, cb * 8, v);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            bytes |= (uint64_t)code1(v[e], hi[e], lo[e]) << (8 * e + k);
+        }
+      }
+      *reinterpret_cast<uint64_t*>(cr + (size_t)m * kD) = bytes;
+    }
   }
 }
 
@@ -182,11 +295,11 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) k_pack_octet_k(
     const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
     uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
-  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
+  __shared__ RowStats st;
   const int row = blockIdx.x;
-  fold_stats<T>(part + (size_t)row * S * 2 * kD, S, 1, blockIdx.y == 0, row, s_alpha, s_beta, s_inv, alpha_out,
+  fold_stats<T>(part + (size_t)row * S * 2 * kD, S, 1, blockIdx.y == 0, row, st, alpha_out,
                 scale_out);
-  k_pack_octet_k_tile<T>(x, n, row, blockIdx.y, tile_tokens, s_alpha, s_beta, s_inv, codes);
+  k_pack_octet_k_tile<T>(GlobalRows<T>{x + (size_t)row * n * kD}, n, row, blockIdx.y, tile_tokens, st, codes);
 }
 
 // OCTET_V layout (bits = 1): channel j's 32-byte row of a 256-token layout
@@ -199,12 +312,12 @@ __global__ void __launch_bounds__(kThreads) k_pack_octet_k(
 // shared memory (rows padded to 9 words, which keeps both the assembly and the
 // read-out within two-to-four-way bank conflicts) and written out with
 // coalesced 4-byte stores.
-template <typename T>
-__device__ __forceinline__ void k_pack_octet_v_tile(const T* __restrict__ x, int n, int row, int tile, int tile_tokens,
-    const float* s_alpha, const float* s_beta, const float* s_inv, uint8_t* __restrict__ codes) {
+template <typename T, typename Src>
+__device__ __forceinline__ void k_pack_octet_v_tile(const Src& src, int n, int row, int tile, int tile_tokens,
+    const RowStats& st, uint8_t* __restrict__ codes) {
   __shared__ float s_hi[kD], s_lo[kD];  // alpha + beta per channel as an exact pair
   __shared__ uint32_t stage[kD * 9];    // [channel][word 0..7, padding]
-  if (threadIdx.x < kD) two_sum(s_alpha[threadIdx.x], s_beta[threadIdx.x], s_hi[threadIdx.x], s_lo[threadIdx.x]);
+  if (threadIdx.x < kD) two_sum(st.alpha[threadIdx.x], st.beta[threadIdx.x], s_hi[threadIdx.x], s_lo[threadIdx.x]);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, cg = lane & 15, hh = lane >> 4;
   float hi[8], lo[8];
@@ -215,25 +328,50 @@ __device__ __forceinline__ void k_pack_octet_v_tile(const T* __restrict__ x, int
   }
   const int n_pad = (n + 255) / 256 * 256;
   const int v0 = tile * (tile_tokens / 256), v1 = min(n_pad / 256, v0 + tile_tokens / 256);
-  const T* xr = x + (size_t)row * n * kD + 8 * cg;
   uint8_t* cr = codes + (size_t)row * (n_pad / 256) * 4096;
+  uint32_t th[4];  // binary16 rows: thresholds of channel pairs (8 cg + 2p, 8 cg + 2p + 1)
+  if constexpr (std::is_same<T, half>::value) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) th[p] = st.thr[8 * cg + 2 * p] | ((uint32_t)st.thr[8 * cg + 2 * p + 1] << 16);
+  }
   for (int vt = v0; vt < v1; ++vt) {
     const int tok0 = vt * 256 + 32 * warp + 16 * hh;
-    uint32_t acc[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // bit i: token tok0 + i
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if (tok0 + i < n) {
-        float v[8];
-        load8(xr + (size_t)(tok0 + i) * kD, v);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] |= code1(v[e], hi[e], lo[e]) << i;
-      }
-    }
     uint32_t word[8];
+    if constexpr (std::is_same<T, half>::value) {
+      // acc[p]: bit i = token tok0 + i of channel 8 cg + 2p, bit 16 + i of channel 8 cg + 2p + 1
+      uint32_t acc[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const uint32_t other = __shfl_xor_sync(0xffffffffu, acc[e], 16);
-      word[e] = hh ? (other | (acc[e] << 16)) : (acc[e] | (other << 16));
+      for (int i = 0; i < 16; ++i) {
+        if (tok0 + i < n) {
+          uint32_t w[4];
+          src.load8h(tok0 + i, 8 * cg, w);
+#pragma unroll
+          for (int p = 0; p < 4; ++p) acc[p] |= ge_mask(w[p], th[p]) & (0x00010001u << i);
+        }
+      }
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const uint32_t other = __shfl_xor_sync(0xffffffffu, acc[p], 16);
+        const uint32_t first = hh ? other : acc[p], second = hh ? acc[p] : other;  // tokens 0..15, 16..31
+        word[2 * p] = __byte_perm(first, second, 0x5410);
+        word[2 * p + 1] = __byte_perm(first, second, 0x7632);
+      }
+    } else {
+      uint32_t acc[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // bit i: token tok0 + i
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (tok0 + i < n) {
+          float v[8];
+          src.load8(tok0 + i, 8 * cg, v);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] |= code1(v[e], hi[e], lo[e]) << i;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t other = __shfl_xor_sync(0xffffffffu, acc[e], 16);
+        word[e] = hh ? (other | (acc[e] << 16)) : (acc[e] | (other << 16));
+      }
     }
     // lane (cg, hh) stores channels 8 cg + 4 hh .. 8 cg + 4 hh + 3
 #pragma unroll
@@ -253,32 +391,31 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) k_pack_octet_v(
     const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
     uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
-  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
+  __shared__ RowStats st;
   const int row = blockIdx.x;
-  fold_stats<T>(part + (size_t)row * S * 2 * kD, S, 1, blockIdx.y == 0, row, s_alpha, s_beta, s_inv, alpha_out,
+  fold_stats<T>(part + (size_t)row * S * 2 * kD, S, 1, blockIdx.y == 0, row, st, alpha_out,
                 scale_out);
-  k_pack_octet_v_tile<T>(x, n, row, blockIdx.y, tile_tokens, s_alpha, s_beta, s_inv, codes);
+  k_pack_octet_v_tile<T>(GlobalRows<T>{x + (size_t)row * n * kD}, n, row, blockIdx.y, tile_tokens, st, codes);
 }
 
 // OCTET_K layout with BITS in {2, 4, 8}: P = 8 / BITS tokens share a byte; a
 // thread owns one byte group (P tokens) x 8 channels, i.e. 8 consecutive bytes.
-template <typename T, int BITS>
-__device__ __forceinline__ void k_pack_octet_k_b_tile(const T* __restrict__ x, int n, int row, int tile, int tile_tokens,
-    const float* s_alpha, const float* s_beta, const float* s_inv, uint8_t* __restrict__ codes) {
+template <typename T, int BITS, typename Src>
+__device__ __forceinline__ void k_pack_octet_k_b_tile(const Src& src, int n, int row, int tile, int tile_tokens,
+    const RowStats& st, uint8_t* __restrict__ codes) {
   constexpr int L = (1 << BITS) - 1, P = 8 / BITS;
   const int cb = threadIdx.x % kTpr, r = threadIdx.x / kTpr;
   float af[8], inv[8];
   double ad[8], bd[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    af[e] = s_alpha[cb * 8 + e];
-    inv[e] = s_inv[cb * 8 + e];
+    af[e] = st.alpha[cb * 8 + e];
+    inv[e] = st.inv[cb * 8 + e];
     ad[e] = (double)af[e];
-    bd[e] = (double)s_beta[cb * 8 + e];
+    bd[e] = (double)st.beta[cb * 8 + e];
   }
   const int groups = (n + P - 1) / P;
   const int m0 = tile * (tile_tokens / P), m1 = min(groups, m0 + tile_tokens / P);
-  const T* xr = x + (size_t)row * n * kD + cb * 8;
   uint8_t* cr = codes + (size_t)row * groups * kD + cb * 8;
   for (int m = m0 + r; m < m1; m += kRpi) {
     uint64_t bytes = 0;
@@ -287,7 +424,7 @@ __device__ __forceinline__ void k_pack_octet_k_b_tile(const T* __restrict__ x, i
       const int i = P * m + k;
       if (i < n) {
         float v[8];
-        load8(xr + (size_t)i * kD, v);
+        src.load8(i, cb * 8, v);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           bytes |= (uint64_t)quant_code(v[e], af[e], inv[e], ad[e], bd[e], L) << (8 * e + BITS * k);
@@ -301,24 +438,23 @@ template <typename T, int BITS>
 __global__ void __launch_bounds__(kThreads) k_pack_octet_k_b(
     const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
     uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
-  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
+  __shared__ RowStats st;
   const int row = blockIdx.x;
-  fold_stats<T>(part + (size_t)row * S * 2 * kD, S, (1 << BITS) - 1, blockIdx.y == 0, row, s_alpha, s_beta, s_inv, alpha_out,
+  fold_stats<T>(part + (size_t)row * S * 2 * kD, S, (1 << BITS) - 1, blockIdx.y == 0, row, st, alpha_out,
                 scale_out);
-  k_pack_octet_k_b_tile<T, BITS>(x, n, row, blockIdx.y, tile_tokens, s_alpha, s_beta, s_inv, codes);
+  k_pack_octet_k_b_tile<T, BITS>(GlobalRows<T>{x + (size_t)row * n * kD}, n, row, blockIdx.y, tile_tokens, st, codes);
 }
 
 // OCTET_V layout with BITS in {2, 4, 8}: tiles of 32 P tokens; byte column q of
 // a tile holds tokens P q .. P q + P - 1. A warp owns one tile: lane q builds
 // byte column q of every channel (consecutive lanes write consecutive bytes).
-template <typename T, int BITS>
-__device__ __forceinline__ void k_pack_octet_v_b_tile(const T* __restrict__ x, int n, int row, int tile, int tile_tokens,
-    const float* s_alpha, const float* s_beta, const float* s_inv, uint8_t* __restrict__ codes) {
+template <typename T, int BITS, typename Src>
+__device__ __forceinline__ void k_pack_octet_v_b_tile(const Src& src, int n, int row, int tile, int tile_tokens,
+    const RowStats& st, uint8_t* __restrict__ codes) {
   constexpr int L = (1 << BITS) - 1, P = 8 / BITS, kTile = 32 * P;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int tiles = (n + kTile - 1) / kTile;
   const int v0 = tile * (tile_tokens / kTile), v1 = min(tiles, v0 + tile_tokens / kTile);
-  const T* xr = x + (size_t)row * n * kD;
   uint8_t* cr = codes + (size_t)row * tiles * 4096;
   for (int vt = v0 + warp; vt < v1; vt += kThreads / 32) {
 #pragma unroll 1
@@ -329,11 +465,11 @@ __device__ __forceinline__ void k_pack_octet_v_b_tile(const T* __restrict__ x, i
         const int i = vt * kTile + P * lane + k;
         if (i < n) {
           float v[8];
-          load8(xr + (size_t)i * kD + cg * 8, v);
+          src.load8(i, cg * 8, v);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int j = cg * 8 + e;
-            bytes[e] |= (uint32_t)quant_code(v[e], s_alpha[j], s_inv[j], (double)s_alpha[j], (double)s_beta[j], L)
+            bytes[e] |= (uint32_t)quant_code(v[e], st.alpha[j], st.inv[j], (double)st.alpha[j], (double)st.beta[j], L)
                         << (BITS * k);
           }
         }
@@ -348,11 +484,11 @@ template <typename T, int BITS>
 __global__ void __launch_bounds__(kThreads) k_pack_octet_v_b(
     const T* __restrict__ x, int n, int S, int tile_tokens, const float* __restrict__ part,
     uint8_t* __restrict__ codes, T* __restrict__ alpha_out, T* __restrict__ scale_out) {
-  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
+  __shared__ RowStats st;
   const int row = blockIdx.x;
-  fold_stats<T>(part + (size_t)row * S * 2 * kD, S, (1 << BITS) - 1, blockIdx.y == 0, row, s_alpha, s_beta, s_inv, alpha_out,
+  fold_stats<T>(part + (size_t)row * S * 2 * kD, S, (1 << BITS) - 1, blockIdx.y == 0, row, st, alpha_out,
                 scale_out);
-  k_pack_octet_v_b_tile<T, BITS>(x, n, row, blockIdx.y, tile_tokens, s_alpha, s_beta, s_inv, codes);
+  k_pack_octet_v_b_tile<T, BITS>(GlobalRows<T>{x + (size_t)row * n * kD}, n, row, blockIdx.y, tile_tokens, st, codes);
 }
 
 // Single-read fill: one thread-block cluster per row, one CTA per tile of
@@ -365,27 +501,48 @@ __global__ void __launch_bounds__(kThreads) k_pack_octet_v_b(
 // that the tiles in flight stay well inside L2, and HBM sees the input once.
 constexpr int kFillMaxCl = 16;
 
+template <typename T, int BITS, int LAYOUT, typename Src>
+__device__ __forceinline__ void pack_tile(const Src& src, int n, int row, int tile, int tile_tokens,
+                                          const RowStats& st,
+                                          uint8_t* __restrict__ codes) {
+  if constexpr (LAYOUT == CQ_LAYOUT_CANONICAL) {
+    k_pack_canonical_tile<T, BITS>(src, n, row, tile, tile_tokens, st, codes);
+  } else if constexpr (LAYOUT == CQ_LAYOUT_OCTET_K) {
+    if constexpr (BITS == 1)
+      k_pack_octet_k_tile<T>(src, n, row, tile, tile_tokens, st, codes);
+    else
+      k_pack_octet_k_b_tile<T, BITS>(src, n, row, tile, tile_tokens, st, codes);
+  } else {
+    if constexpr (BITS == 1)
+      k_pack_octet_v_tile<T>(src, n, row, tile, tile_tokens, st, codes);
+    else
+      k_pack_octet_v_b_tile<T, BITS>(src, n, row, tile, tile_tokens, st, codes);
+  }
+}
+
 template <typename T, int BITS, int LAYOUT>
 __global__ void __launch_bounds__(kThreads, 4) k_fill(const T* __restrict__ x, int n, int cl, int tile_tokens,
-                                                   uint8_t* __restrict__ codes, T* __restrict__ alpha_out,
-                                                   T* __restrict__ scale_out) {
+                                                      uint8_t* __restrict__ codes, T* __restrict__ alpha_out,
+                                                      T* __restrict__ scale_out) {
+  __shared__ float smn[kRpi][kD], smx[kRpi][kD];
   __shared__ float recv[kFillMaxCl][2][kD];  // every CTA's (min, max) per channel
-  __shared__ float s_alpha[kD], s_beta[kD], s_inv[kD];
+  __shared__ RowStats st;
   const uint32_t rank = tc::cluster_rank();
   const int row = blockIdx.x / cl;
   tc::cluster_arrive_relaxed();  // matched by the wait before the first peer store
   const int i0 = (int)rank * tile_tokens, i1 = min(n, i0 + tile_tokens);
+  const T* xrow = x + (size_t)row * n * kD;
   {
     // the whole tile is requested into L2 at once (16 KB per request), so HBM
     // sees every resident CTA's tile in flight; both passes below read from L2
     constexpr int kReq = 16 * 1024;
-    const char* tile0 = reinterpret_cast<const char*>(x + ((size_t)row * n + i0) * kD);
+    const char* tile0 = reinterpret_cast<const char*>(xrow + (size_t)i0 * kD);
     const int bytes = (i1 - i0) * kD * (int)sizeof(T);
     if ((int)threadIdx.x * kReq < bytes)
       tc::prefetch_l2_bulk(tile0 + (size_t)threadIdx.x * kReq, (uint32_t)min(kReq, bytes - (int)threadIdx.x * kReq));
   }
   float a, b;
-  tile_minmax<T>(x + (size_t)row * n * kD, i0, i1, a, b);
+  tile_minmax<T>(xrow, i0, i1, a, b, smn, smx);
   tc::cluster_wait();  // every CTA of the cluster is running
   if (threadIdx.x < kD) {
     for (int r = 0; r < cl; ++r) {
@@ -395,21 +552,8 @@ __global__ void __launch_bounds__(kThreads, 4) k_fill(const T* __restrict__ x, i
   }
   tc::cluster_sync();  // every partial has landed; no peer access after this point
   constexpr int L = (1 << BITS) - 1;
-  fold_stats<T>(&recv[0][0][0], cl, L, rank == 0, row, s_alpha, s_beta, s_inv, alpha_out, scale_out);
-  const int tile = (int)rank;
-  if constexpr (LAYOUT == CQ_LAYOUT_CANONICAL) {
-    k_pack_canonical_tile<T, BITS>(x, n, row, tile, tile_tokens, s_alpha, s_beta, s_inv, codes);
-  } else if constexpr (LAYOUT == CQ_LAYOUT_OCTET_K) {
-    if constexpr (BITS == 1)
-      k_pack_octet_k_tile<T>(x, n, row, tile, tile_tokens, s_alpha, s_beta, s_inv, codes);
-    else
-      k_pack_octet_k_b_tile<T, BITS>(x, n, row, tile, tile_tokens, s_alpha, s_beta, s_inv, codes);
-  } else {
-    if constexpr (BITS == 1)
-      k_pack_octet_v_tile<T>(x, n, row, tile, tile_tokens, s_alpha, s_beta, s_inv, codes);
-    else
-      k_pack_octet_v_b_tile<T, BITS>(x, n, row, tile, tile_tokens, s_alpha, s_beta, s_inv, codes);
-  }
+  fold_stats<T>(&recv[0][0][0], cl, L, rank == 0, row, st, alpha_out, scale_out);
+  pack_tile<T, BITS, LAYOUT>(GlobalRows<T>{xrow}, n, row, (int)rank, tile_tokens, st, codes);
 }
 
 // Tile of the single-read fill for a row of n tokens (0: not supported, use
