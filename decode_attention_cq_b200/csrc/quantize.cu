@@ -303,60 +303,72 @@ __global__ void __launch_bounds__(kThreads) k_pack_octet_k(
 }
 
 // OCTET_V layout (bits = 1): channel j's 32-byte row of a 256-token layout
-// tile is the 256-bit vector of its codes in token order. The CTA takes its
-// tile 256 tokens at a time; warp w owns tokens 32 w .. 32 w + 31, i.e. word w
-// of every channel's row. Lane l reads channels 8 (l % 16) .. + 7 of tokens
-// 16 (l / 16) .. + 15 (so each load instruction covers two whole token rows),
-// sets one bit per token in a 16-bit word per channel, and the two half-warps
-// join their halves with one exchange. The 4 KB layout tile is assembled in
-// shared memory (rows padded to 9 words, which keeps both the assembly and the
-// read-out within two-to-four-way bank conflicts) and written out with
-// coalesced 4-byte stores.
+// tile is the 256-bit vector of its codes in token order (byte o = tokens
+// 8 o .. 8 o + 7). The CTA takes its tile 256 tokens at a time and assembles
+// each 4 KB layout tile in shared memory (rows padded to 9 words), then writes
+// it out with coalesced 4-byte stores.
+//  - binary16: a thread takes one octet x 8 channels at a time, like the
+//    octet-K pack (each load instruction of a warp covers two token rows), and
+//    drops its 8 channel bytes into the staged tile;
+//  - binary32: warp w owns tokens 32 w .. 32 w + 31, i.e. word w of every
+//    channel's row. Lane l reads channels 8 (l % 16) .. + 7 of tokens
+//    16 (l / 16) .. + 15, sets one bit per token in a 16-bit word per channel,
+//    and the two half-warps join their halves with one exchange.
 template <typename T, typename Src>
 __device__ __forceinline__ void k_pack_octet_v_tile(const Src& src, int n, int row, int tile, int tile_tokens,
     const RowStats& st, uint8_t* __restrict__ codes) {
-  __shared__ float s_hi[kD], s_lo[kD];  // alpha + beta per channel as an exact pair
-  __shared__ uint32_t stage[kD * 9];    // [channel][word 0..7, padding]
-  if (threadIdx.x < kD) two_sum(st.alpha[threadIdx.x], st.beta[threadIdx.x], s_hi[threadIdx.x], s_lo[threadIdx.x]);
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, cg = lane & 15, hh = lane >> 4;
-  float hi[8], lo[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    hi[e] = s_hi[8 * cg + e];
-    lo[e] = s_lo[8 * cg + e];
-  }
+  __shared__ uint32_t stage[kD * 9];  // [channel][word 0..7, padding]
   const int n_pad = (n + 255) / 256 * 256;
   const int v0 = tile * (tile_tokens / 256), v1 = min(n_pad / 256, v0 + tile_tokens / 256);
   uint8_t* cr = codes + (size_t)row * (n_pad / 256) * 4096;
-  uint32_t th[4];  // binary16 rows: thresholds of channel pairs (8 cg + 2p, 8 cg + 2p + 1)
   if constexpr (std::is_same<T, half>::value) {
+    uint8_t* sb = reinterpret_cast<uint8_t*>(stage);
+    const int cg = threadIdx.x % kTpr, r = threadIdx.x / kTpr;
+    uint32_t th[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) th[p] = st.thr[8 * cg + 2 * p] | ((uint32_t)st.thr[8 * cg + 2 * p + 1] << 16);
-  }
-  for (int vt = v0; vt < v1; ++vt) {
-    const int tok0 = vt * 256 + 32 * warp + 16 * hh;
-    uint32_t word[8];
-    if constexpr (std::is_same<T, half>::value) {
-      // acc[p]: bit i = token tok0 + i of channel 8 cg + 2p, bit 16 + i of channel 8 cg + 2p + 1
-      uint32_t acc[4] = {0u, 0u, 0u, 0u};
+    for (int vt = v0; vt < v1; ++vt) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        if (tok0 + i < n) {
-          uint32_t w[4];
-          src.load8h(tok0 + i, 8 * cg, w);
+      for (int oo = 0; oo < 2; ++oo) {
+        const int o = r + kRpi * oo, tok0 = vt * 256 + 8 * o;  // octet o of the layout tile
+        uint32_t acc[4] = {0u, 0u, 0u, 0u};  // bit k / 16 + k: token tok0 + k of channel 8 cg + 2p / + 1
 #pragma unroll
-          for (int p = 0; p < 4; ++p) acc[p] |= ge_mask(w[p], th[p]) & (0x00010001u << i);
+        for (int k = 0; k < 8; ++k) {
+          if (tok0 + k < n) {
+            uint32_t w[4];
+            src.load8h(tok0 + k, 8 * cg, w);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) acc[p] |= ge_mask(w[p], th[p]) & (0x00010001u << k);
+          }
+        }
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          sb[(8 * cg + 2 * p) * 36 + o] = (uint8_t)acc[p];
+          sb[(8 * cg + 2 * p + 1) * 36 + o] = (uint8_t)(acc[p] >> 16);
         }
       }
+      __syncthreads();
+      uint32_t* dst = reinterpret_cast<uint32_t*>(cr + (size_t)vt * 4096);
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const uint32_t other = __shfl_xor_sync(0xffffffffu, acc[p], 16);
-        const uint32_t first = hh ? other : acc[p], second = hh ? acc[p] : other;  // tokens 0..15, 16..31
-        word[2 * p] = __byte_perm(first, second, 0x5410);
-        word[2 * p + 1] = __byte_perm(first, second, 0x7632);
+      for (int k = 0; k < 4; ++k) {
+        const int w = (int)threadIdx.x + kThreads * k;  // word w: channel w / 8, word w % 8 of its row
+        dst[w] = stage[(w >> 3) * 9 + (w & 7)];
       }
-    } else {
+      __syncthreads();
+    }
+  } else {
+    __shared__ float s_hi[kD], s_lo[kD];  // alpha + beta per channel as an exact pair
+    if (threadIdx.x < kD) two_sum(st.alpha[threadIdx.x], st.beta[threadIdx.x], s_hi[threadIdx.x], s_lo[threadIdx.x]);
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, cg = lane & 15, hh = lane >> 4;
+    float hi[8], lo[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      hi[e] = s_hi[8 * cg + e];
+      lo[e] = s_lo[8 * cg + e];
+    }
+    for (int vt = v0; vt < v1; ++vt) {
+      const int tok0 = vt * 256 + 32 * warp + 16 * hh;
       uint32_t acc[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // bit i: token tok0 + i
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -367,23 +379,24 @@ __device__ __forceinline__ void k_pack_octet_v_tile(const Src& src, int n, int r
           for (int e = 0; e < 8; ++e) acc[e] |= code1(v[e], hi[e], lo[e]) << i;
         }
       }
+      uint32_t word[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const uint32_t other = __shfl_xor_sync(0xffffffffu, acc[e], 16);
         word[e] = hh ? (other | (acc[e] << 16)) : (acc[e] | (other << 16));
       }
-    }
-    // lane (cg, hh) stores channels 8 cg + 4 hh .. 8 cg + 4 hh + 3
+      // lane (cg, hh) stores channels 8 cg + 4 hh .. 8 cg + 4 hh + 3
 #pragma unroll
-    for (int j = 0; j < 4; ++j) stage[(8 * cg + 4 * hh + j) * 9 + warp] = hh ? word[4 + j] : word[j];
-    __syncthreads();
-    uint32_t* dst = reinterpret_cast<uint32_t*>(cr + (size_t)vt * 4096);
+      for (int j2 = 0; j2 < 4; ++j2) stage[(8 * cg + 4 * hh + j2) * 9 + warp] = hh ? word[4 + j2] : word[j2];
+      __syncthreads();
+      uint32_t* dst = reinterpret_cast<uint32_t*>(cr + (size_t)vt * 4096);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int w = (int)threadIdx.x + kThreads * k;  // word w: channel w / 8, word w % 8 of its row
-      dst[w] = stage[(w >> 3) * 9 + (w & 7)];
+      for (int k = 0; k < 4; ++k) {
+        const int w = (int)threadIdx.x + kThreads * k;  // word w: channel w / 8, word w % 8 of its row
+        dst[w] = stage[(w >> 3) * 9 + (w & 7)];
+      }
+      __syncthreads();
     }
-    __syncthreads();
   }
 }
 
@@ -524,9 +537,13 @@ template <typename T, int BITS, int LAYOUT>
 __global__ void __launch_bounds__(kThreads, 4) k_fill(const T* __restrict__ x, int n, int cl, int tile_tokens,
                                                       uint8_t* __restrict__ codes, T* __restrict__ alpha_out,
                                                       T* __restrict__ scale_out) {
-  __shared__ float smn[kRpi][kD], smx[kRpi][kD];
+  // dynamic: the per-row-group min / max of pass 1 (also what pads the CTA's
+  // shared memory to the residency cap)
+  extern __shared__ __align__(128) uint8_t fill_dyn[];
   __shared__ float recv[kFillMaxCl][2][kD];  // every CTA's (min, max) per channel
   __shared__ RowStats st;
+  float(*smn)[kD] = reinterpret_cast<float(*)[kD]>(fill_dyn + ((128u - (tc::smem_u32(fill_dyn) & 127u)) & 127u));
+  float(*smx)[kD] = smn + kRpi;
   const uint32_t rank = tc::cluster_rank();
   const int row = blockIdx.x / cl;
   tc::cluster_arrive_relaxed();  // matched by the wait before the first peer store
@@ -568,12 +585,13 @@ template <typename T, int BITS, int LAYOUT>
 cudaError_t launch_fill(const T* x, int rows, int n, uint8_t* codes, T* alpha, T* scale, cudaStream_t stream) {
   const int tile = fill_tile_tokens(n);
   const int cl = (n + tile - 1) / tile;
-  // Dynamic shared memory only to cap residency at 4 CTAs per SM: 4 x 148 tiles
-  // of 512 tokens x 256 B = 76 MB in flight, inside the 126 MB L2, so each
-  // tile's second read hits L2 (at 1024-token tiles the cap is the same). The
-  // pad brings static + dynamic to 46 KB: more than 228 KB / 5, and within the
-  // 48 KB a launch may use without opting in.
+  // Dynamic shared memory: the pass-1 scratch, padded to cap residency at 4 CTAs
+  // per SM: 4 x 148 tiles of 512 tokens x 256 B = 76 MB in flight, inside the
+  // 126 MB L2, so each tile's second read hits L2 (at 1024-token tiles the cap
+  // is the same). Static + dynamic = 46 KB: more than 228 KB / 5, and within
+  // the 48 KB a launch may use without opting in.
   constexpr int kTotal = 46 * 1024;
+  constexpr int kScratch = 2 * kRpi * kD * (int)sizeof(float) + 128;  // + alignment
   static int pads[kMaxDevices];  // per device, + 1 once set (benign race: every caller computes the same values)
   const int dev = current_device();
   if (dev < 0) return cudaErrorInvalidDevice;
@@ -582,7 +600,8 @@ cudaError_t launch_fill(const T* x, int rows, int n, uint8_t* codes, T* alpha, T
     cudaFuncAttributes fa;
     if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, k_fill<T, BITS, LAYOUT>);
     if (e != cudaSuccess) return e;
-    pads[dev] = 1 + (fa.sharedSizeBytes < (size_t)kTotal ? kTotal - (int)fa.sharedSizeBytes : 0);
+    const int pad = (int)fa.sharedSizeBytes + kScratch < kTotal ? kTotal - (int)fa.sharedSizeBytes : kScratch;
+    pads[dev] = 1 + pad;
   }
   const int pad = pads[dev] - 1;
   cudaLaunchConfig_t cfg = {};
