@@ -726,6 +726,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int s = 0; s < kSlots; ++s)
       if (F.uses[s] > 0) tc::mbar_wait(&F.full[s], (F.uses[s] - 1) & 1u, kSpin);
   }
+  // The split launch starts while the whole rows still run; it does not finish
+  // before them, so that work after the decode on the stream sees all rows.
+  if constexpr (kSplit) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // Tensor-memory columns for a CTA's tiles: 32 per tile of a lane quarter, a

@@ -119,3 +119,26 @@ def test_row_kernel_split_rows(row_kernel, n):
         ref = oracle.decode_attention(f64(q[sl]), f64(k[sl]), f64(v[sl]), 1, "f16", calib)["out"]
         err = row_rel_err(out[sl].float().numpy(), ref_output_rounded(ref, torch.float16))
         assert err <= OUT_RTOL, (n, b, err)
+
+
+def test_split_rows_are_ordered_before_later_stream_work(row_kernel):
+    """The split rows start while the whole rows still run (a programmatic
+    dependent launch), yet work queued after the call on the same stream must
+    see every row: a device copy and a host copy taken right after the call,
+    with no synchronization in between, equal the output read after it."""
+    Bb, Hkv, n = 40, 8, 8192  # 320 rows: 24 of them run split on B200
+    K, V = cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V
+    assert cq.cq_decode_launch_count(K, V, Bb, 4 * Hkv, Hkv, n, 128, 1) == 2
+    q, k, v = synth.make_case(Bb, 4 * Hkv, Hkv, n, 128, "f16", outliers=4, seed=77, device=row_kernel)
+    kq, vq = _quant(k, v, row_kernel)
+    out = torch.empty_like(q)
+    host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    for _ in range(5):
+        out.fill_(float("nan"))
+        cq.cq_decode_attn(q, kq, vq, calib=CALIBS[1], out=out)
+        snap = out.clone()
+        host.copy_(out, non_blocking=True)
+        torch.cuda.synchronize()
+        assert not torch.isnan(out).any()
+        assert torch.equal(snap, out)
+        assert torch.equal(host, out.cpu())
