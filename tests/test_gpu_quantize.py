@@ -180,3 +180,53 @@ def test_one_bit_f32_codes_across_fill_limits(cuda_device, n):
         qc = cq.cq_quantize_kv(x.to(cuda_device), 1, layout)
         torch.cuda.synchronize()
         _check_quantized(x, qc, 1, layout)
+
+
+def test_one_bit_f16_thresholds_at_zero_subnormals_and_extremes(cuda_device):
+    """Binary16 1-bit codes are decided against the smallest binary16 above the
+    channel midpoint mu = (alpha + beta) / 2. Every way of finding it is met:
+    - mu = 0, where the threshold is the smallest subnormal;
+    - mu between -2^-24 and 0, and between 0 and 2^-24;
+    - mu an exact negative subnormal, where one step up reaches -0;
+    - mu halfway between subnormals;
+    - mu halfway between the two largest finite values;
+    - a constant channel at 65504, where the threshold is +inf;
+    - mu = 0 with both signed zeros among the tokens.
+    Codes, alpha and step are compared bit-exactly with the oracle in every
+    layout, with a ragged token count."""
+    f = np.float16
+    sub = lambda k: f(k * 2.0 ** -24)  # noqa: E731  (k times the smallest subnormal)
+    cases = [  # (alpha, beta, tokens inside [alpha, beta] that must appear)
+        (f(-1), f(1), [f(0), f(-0.0), sub(1), -sub(1), sub(3), -sub(2)]),
+        (-sub(1), sub(2), [f(0), f(-0.0), sub(1)]),
+        (-sub(2), sub(1), [f(0), f(-0.0), -sub(1)]),
+        (-sub(3), sub(1), [-sub(1), -sub(2), f(-0.0), f(0)]),
+        (sub(3), sub(8), [sub(4), sub(5), sub(6), sub(7)]),
+        (f(65472), f(65504), []),
+        (f(-65504), f(65504), [f(0), f(-0.0), sub(1), -sub(1), f(65472), f(-65472)]),
+        (f(65504), f(65504), []),
+        (f(-2.0 ** -14), f(2.0 ** -14), [sub(1), -sub(1), f(0), f(-0.0), sub(1023), -sub(1023)]),
+    ]
+    rng = np.random.default_rng(5)
+    n, d = 77, 128
+    x = np.zeros((1, 2, n, d), dtype=f)
+    for c in range(d):
+        a, b, extra = cases[c % len(cases)]
+        mid = (float(a) + float(b)) / 2.0  # exact in double
+        near = [f(mid)]
+        for step in (np.inf, -np.inf):
+            v = f(mid)
+            for _ in range(3):
+                v = np.nextafter(v, f(step), dtype=f)
+                near.append(v)
+        near = [v for v in near if a <= v <= b and np.isfinite(v)]
+        vals = [a, b] + extra + near
+        rest = rng.uniform(float(a), float(b), n - len(vals)).astype(f)
+        col = np.array(vals + list(rest), dtype=f)
+        x[0, 0, :, c] = col
+        x[0, 1, :, c] = col[rng.permutation(n)]
+    xt = torch.from_numpy(x)
+    for layout in (cq.LAYOUT_CANONICAL, cq.LAYOUT_OCTET_K, cq.LAYOUT_OCTET_V):
+        qc = cq.cq_quantize_kv(xt.to(cuda_device), 1, layout)
+        torch.cuda.synchronize()
+        _check_quantized(xt, qc, 1, layout)
