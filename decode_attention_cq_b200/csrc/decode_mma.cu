@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk)
 #pragma unroll
-        for (int tl = 0; tl < 2; ++tl) d[kk][tl][0] = d[kk][tl][1] = d[kk][tl][2] = d[kk][tl][3] = kAccBias;
+        for (int tl = 0; tl < 2; ++tl) d[kk][tl][0] = d[kk][tl][1] = d[kk][tl][2] = d[kk][tl][3] = 0;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
@@ -240,9 +240,8 @@ __global__ void __launch_bounds__(kThreads, S == 2048 ? 3 : 1)
         const float sc = kscale * __int_as_float((127 - k - kk) << 23);  // step * 2^-k
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          // limb sums read back from their biased accumulators (|D| < 2^22)
-          const float v = fmaf(16384.f, acc_value(d[kk][1][2 * r]),
-                               fmaf(128.f, acc_value(d[kk][0][2 * r + 1]), acc_value(d[kk][0][2 * r])));
+          const int d01 = d[kk][0][2 * r] + (d[kk][0][2 * r + 1] << 7);  // |d01| < 2^29
+          const float v = fmaf(16384.f, (float)d[kk][1][2 * r], (float)d01);
           const float x = fmaf(v, sc, c0);
           if (tok + 64 * r + k + kk < t1) {
             mn = fminf(mn, x);

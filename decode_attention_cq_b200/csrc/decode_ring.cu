@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, ring_slots<BITS>() == 2 ? 3 : 2)
 #pragma unroll
         for (int kk = 0; kk < KK; ++kk)
 #pragma unroll
-          for (int tl = 0; tl < 2; ++tl) d[kk][tl][0] = d[kk][tl][1] = d[kk][tl][2] = d[kk][tl][3] = kAccBias;
+          for (int tl = 0; tl < 2; ++tl) d[kk][tl][0] = d[kk][tl][1] = d[kk][tl][2] = d[kk][tl][3] = 0;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
@@ -266,9 +266,8 @@ __global__ void __launch_bounds__(kThreads, ring_slots<BITS>() == 2 ? 3 : 2)
           const float sc = kscale * __int_as_float((127 - (k + kk) * BITS) << 23);  // step * 2^-(k b)
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
-            // limb sums read back from their biased accumulators (|D| < 2^22)
-            const float v = fmaf(16384.f, acc_value(d[kk][1][2 * r]),
-                                 fmaf(128.f, acc_value(d[kk][0][2 * r + 1]), acc_value(d[kk][0][2 * r])));
+            const int d01 = d[kk][0][2 * r] + (d[kk][0][2 * r + 1] << 7);  // |d01| < 2^30
+            const float v = fmaf(16384.f, (float)d[kk][1][2 * r], (float)d01);
             const float x = fmaf(v, sc, c0);
             if (full || tok + 8 * P * r + k + kk < t1) {
               mn = fminf(mn, x);

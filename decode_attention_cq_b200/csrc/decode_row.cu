@@ -370,15 +370,10 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int kp = 0; kp < 4; ++kp) {
         int d[2][4][4];  // [bit 2 kp + kk][N tile][reg]
-        // Every accumulator starts at the bit pattern of 1.5 * 2^23. A limb sum has
-        // |D| <= 128 channels x 128 x 2^7 = 2^21 < 2^22, so the integer adds keep
-        // the exponent field and the word reads back as the float 1.5 * 2^23 + D:
-        // one subtraction recovers D exactly, with no integer-to-float conversion
-        // (a quarter-rate instruction, five of them per logit pair otherwise).
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk)
 #pragma unroll
-          for (int jn = 0; jn < 4; ++jn) d[kk][jn][0] = d[kk][jn][1] = d[kk][jn][2] = d[kk][jn][3] = kAccBias;
+          for (int jn = 0; jn < 4; ++jn) d[kk][jn][0] = d[kk][jn][1] = d[kk][jn][2] = d[kk][jn][3] = 0;
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) {
           const uint32_t msk = 0x01010101u << (2 * kp + kk);
@@ -387,27 +382,25 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int jn = 0; jn < 4; ++jn) mma_s8u8(d[kk][jn], wa[cc], bk[cc][jn][0] & msk, bk[cc][jn][1] & msk);
         }
-        // lo lanes finish bit 2 kp, hi lanes bit 2 kp + 1: x = D0 + 2^7 D1 + 2^14 D2.
-        // lo lanes hold D0, D2 of both bits, hi lanes D1 (their D2 row is the zero
-        // row, so it reads back as 0): lo sends D0 + 2^14 D2 of bit 2 kp + 1, hi
-        // sends D1 of bit 2 kp. The multipliers pick each lane's operands on the
-        // FMA pipe, which leaves the integer pipe to the code masking.
+        // lo lanes finish bit 2 kp, hi lanes bit 2 kp + 1: x = D0 + 2^7 D1 + 2^14 D2
         const int kown = 2 * kp + (lo ? 0 : 1);
         const float sc = kscale * __int_as_float((127 - kown) << 23);  // step * 2^-k
-        const float m_lo = lo ? 1.f : 0.f, m_hi = lo ? 0.f : 1.f;
-        const float m_recv = lo ? 128.f : 1.f, m_hi128 = lo ? 0.f : 128.f;
         uint32_t out[8];
 #pragma unroll
         for (int jn = 0; jn < 4; ++jn)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int i = 2 * jn + e;
-            const float f00 = acc_value(d[0][jn][e]), f02 = acc_value(d[0][jn][2 + e]);
-            const float f10 = acc_value(d[1][jn][e]), f12 = acc_value(d[1][jn][2 + e]);
-            const float send = fmaf(16384.f, f12, fmaf(m_lo, f10, m_hi * f00));
-            const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-            // lo: 2^7 D1 (received) + D0 + 2^14 D2; hi: 2^7 D1 + (D0 + 2^14 D2) received
-            const float x = fmaf(16384.f, f02, fmaf(m_recv, recv, fmaf(m_lo, f00, m_hi128 * f10)));
+            const int send =
+                lo ? __float_as_int(fmaf(16384.f, (float)d[1][jn][2 + e], (float)d[1][jn][e])) : d[0][jn][e];
+            const int recv = __shfl_xor_sync(0xffffffffu, send, 16);
+            float x;
+            if (lo) {
+              const int d01 = d[0][jn][e] + (recv << 7);  // |d01| < 2^29
+              x = fmaf(16384.f, (float)d[0][jn][2 + e], (float)d01);
+            } else {
+              x = fmaf(128.f, (float)d[1][jn][e], __int_as_float(recv));
+            }
             const float xl = fmaf(x, sc, c0);
             if (!ragged || (have && kTile * jg + 8 * lane_octet(tq, i) + kown < n)) {
               mn = fminf(mn, xl);
@@ -726,9 +719,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int s = 0; s < kSlots; ++s)
       if (F.uses[s] > 0) tc::mbar_wait(&F.full[s], (F.uses[s] - 1) & 1u, kSpin);
   }
-  // The split launch starts while the whole rows still run; it does not finish
-  // before them, so that work after the decode on the stream sees all rows.
-  if constexpr (kSplit) asm volatile("griddepcontrol.wait;" ::: "memory");
+  // The split launch starts while the whole rows still run. Its last CTA (the
+  // last to be scheduled) waits for them before it exits, so the split grid
+  // does not complete before the whole-row grid, and work after the decode on
+  // the stream sees every row; the other CTAs free their SM slots at once.
+  if constexpr (kSplit)
+    if (blockIdx.x == gridDim.x - 1) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // Tensor-memory columns for a CTA's tiles: 32 per tile of a lane quarter, a
@@ -755,9 +751,10 @@ cudaError_t set_row_attributes(size_t smem) {
 }
 
 int device_sms() {
-  static int count[64] = {};  // per device ordinal; 0 until read
-  int dev = 0, c = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  static int count[kMaxDevices] = {};  // per device ordinal; 0 until read
+  const int dev = current_device();
+  int c = 0;
+  if (dev < 0) return 0;
   if (count[dev] == 0 && cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
     count[dev] = c;
   return count[dev];

@@ -16,13 +16,6 @@ namespace mu {
 constexpr int kG = 4;                 // query heads per kv-head
 constexpr uint32_t kSpin = 1u << 24;  // bound on every mbarrier wait (about a second)
 
-// An int32 accumulator that starts at kAccBias (the bit pattern of 1.5 * 2^23)
-// and gains integer d with |d| < 2^22 keeps its exponent field: its bits read
-// as the float 1.5 * 2^23 + d, and acc_value returns d exactly with one float
-// subtraction instead of an integer-to-float conversion.
-constexpr int kAccBias = 0x4B400000;
-__device__ __forceinline__ float acc_value(int acc) { return __int_as_float(acc) - 12582912.0f; }
-
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
