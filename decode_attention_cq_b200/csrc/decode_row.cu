@@ -76,6 +76,13 @@ constexpr int kTile = 256;              // tokens per tile (32 octets, 4 KB of c
 constexpr int kChunkTiles = 4;          // tiles per ring slot
 constexpr int kChunkBytes = kChunkTiles * 4096;
 constexpr int kSlots = 4;
+// The ring's waits are parity waits, so a warp may wait on a slot's next use
+// only once the slot's previous use has landed. Each warp group reuses only
+// the slots of chunks it consumes itself: K chunks alternate between warps
+// 0-3 and 4-7 (slots of one parity each), every warp reads every V chunk (and
+// a CTA barrier separates the two sides), and the two groups take alternate
+// text chunk pairs (two slots each). That needs kSlots to be a multiple of 4.
+static_assert(kSlots % 4 == 0, "warp groups must own their ring slots");
 constexpr int kMaxTiles = 32;  // n <= 8192: 8 tiles per tensor-memory lane quarter, 256 columns
 constexpr int kWMax = (1 << 21) - 1;
 constexpr int kLimbRow = 132;  // bytes per limb row (padding spreads the fragment loads over banks)
