@@ -93,6 +93,11 @@ __global__ void __launch_bounds__(kThreads) k_text_merge(const T* __restrict__ q
 // four warps reading a chunk release it through a shared counter, and the one
 // that completes the count issues the chunk that reuses the slot.
 constexpr int kSlots = 4;
+// Parity waits: a warp may wait on a slot's next use only once its previous
+// use has landed. The two warp groups take alternate chunk pairs (keys, values)
+// from chunk 0, so with a multiple of 4 slots each group reuses only its own
+// two slots.
+static_assert(kSlots % 4 == 0, "warp groups must own their ring slots");
 
 struct TextRing {
   uint64_t full[kSlots];
