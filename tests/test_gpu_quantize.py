@@ -182,6 +182,10 @@ def test_one_bit_f32_codes_across_fill_limits(cuda_device, n):
         _check_quantized(x, qc, 1, layout)
 
 
+# The +-65504 channel: steps past the largest finite value overflow to inf (and
+# are dropped), and its step 131008 is stored as +inf by the oracle and the
+# library alike.
+@np.errstate(over="ignore")
 def test_one_bit_f16_thresholds_at_zero_subnormals_and_extremes(cuda_device):
     """Binary16 1-bit codes are decided against the smallest binary16 above the
     channel midpoint mu = (alpha + beta) / 2. Every way of finding it is met:
