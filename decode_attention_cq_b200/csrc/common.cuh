@@ -17,6 +17,16 @@ inline int current_device() {
   int dev = 0;
   return cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices ? dev : -1;
 }
+// SM count of the current device, read once per device (0 if unknown).
+inline int device_sms() {
+  static int count[kMaxDevices] = {};  // benign race: every caller stores the same value
+  const int dev = current_device();
+  int c = 0;
+  if (dev < 0) return 0;
+  if (count[dev] == 0 && cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+    count[dev] = c;
+  return count[dev];
+}
 
 // ---------------------------------------------------------------- dtypes ----
 template <typename T>

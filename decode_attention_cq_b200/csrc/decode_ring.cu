@@ -17,8 +17,7 @@
 // One thread-block cluster per (batch, kv-head) row, one CTA per 2048-token
 // slice, whatever b is. Only the slice's logits (later its weight fragments,
 // 16 bytes per token) stay resident; the codes (32 b KB per slice for K and
-// again for V) stream through a ring of 16 KB tensor copies (2 slots, 4 for
-// 4- and 8-bit codes): K
+// again for V) stream through a ring of four 16 KB tensor copies: K
 // chunks first, then V chunks, so the first V chunks load while the cluster
 // exchanges the logit range. A slot is refilled once all eight warps have
 // released it (full / empty mbarriers, every wait bounded).
@@ -63,23 +62,26 @@ struct RingFixed {
   float recv[kRecv];                // [src][h][channel - first owned channel]
 };
 
-// Ring slots: 2 (3 CTAs per SM) while the K / V loops have work to hide the
-// copies behind; 4 (2 CTAs per SM, more bytes in flight per SM) for 4- and
-// 8-bit codes, where the kernel mostly waits on its copies.
-template <int BITS>
-constexpr int ring_slots() { return BITS >= 4 ? 4 : 2; }
+// Ring slots (SLOTS): 4 with 2 CTAs per SM (more bytes in flight per CTA), or
+// 2 with 3 CTAs per SM (more CTAs resident). 4- and 8-bit codes, where the
+// kernel mostly waits on its copies, always take 4 (8-bit at batch 16,
+// n = 8192: 78.6 -> 67.8 us). 2-bit codes take 4 while the launch fits in two
+// waves of 2 CTAs per SM, 2 beyond that (measured on B200, n = 8192: batch 16
+// 40.9 -> 37.9 us with 4; batch 32 67.4 -> 62.9 us and batch 64 117.2 ->
+// 103.1 us with 2).
+inline int ring_slots_2bit(long long ctas, int sms) { return sms > 0 && ctas <= 4LL * sms ? 4 : 2; }
 
 // logits / weight fragments (16 B per token) | ring (slots x 16 KB) | fixed part
-template <typename T, int BITS>
+template <typename T, int SLOTS>
 constexpr size_t ring_smem_bytes() {
-  return (size_t)kSlice * 16 + (size_t)ring_slots<BITS>() * kChunkBytes + sizeof(RingFixed<T>);
+  return (size_t)kSlice * 16 + (size_t)SLOTS * kChunkBytes + sizeof(RingFixed<T>);
 }
 
 // kmap: K codes as [rows][byte rows][128 B]; vmap: V codes as [rows][tiles *
 // 32][128 B] (a 128-byte line holds 4 channels' 32 bytes of a tile). Both use
 // the 128-byte swizzle (chunk c of line l lands at chunk c ^ (l & 7)).
-template <typename T, int BITS>
-__global__ void __launch_bounds__(kThreads, ring_slots<BITS>() == 2 ? 3 : 2)
+template <typename T, int BITS, int SLOTS>
+__global__ void __launch_bounds__(kThreads, SLOTS == 2 ? 3 : 2)
     k_decode_ring(const __grid_constant__ DecodeArgs a, int cl, const __grid_constant__ CUtensorMap kmap,
                   const __grid_constant__ CUtensorMap vmap) {
   constexpr int P = 8 / BITS;         // tokens per code byte
@@ -87,7 +89,7 @@ __global__ void __launch_bounds__(kThreads, ring_slots<BITS>() == 2 ? 3 : 2)
   constexpr int kTileTok = 32 * P;    // tokens per V tile (32 byte columns, 4 KB)
   constexpr int kUnitWords = 64 * P;  // logit words per unit (16 byte rows x P x 4 heads)
   constexpr uint32_t kSubMask = 0x01010101u * ((1u << BITS) - 1u);  // sub-position 0 of every byte
-  constexpr int kSlots = ring_slots<BITS>();
+  constexpr int kSlots = SLOTS;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the 128-byte swizzle of the copies repeats every 1024 bytes: align to it
@@ -502,24 +504,19 @@ __global__ void __launch_bounds__(kThreads, ring_slots<BITS>() == 2 ? 3 : 2)
   }
 }
 
-template <typename T, int BITS>
-cudaError_t run_bits(const DecodeArgs& a, cudaStream_t stream) {
-  constexpr int P = 8 / BITS, kTileTok = 32 * P;
-  const int rows = a.B * a.Hkv;
-  const int nvt = (a.n + kTileTok - 1) / kTileTok;
-  const int per = kSlice / kTileTok;  // V tiles per CTA
-  const int cl = (nvt + per - 1) / per;
-  if (cl > kMaxCl || (long long)rows * cl > 0x7fffffffLL) return cudaErrorNotSupported;
-  const size_t smem = ring_smem_bytes<T, BITS>() + 1024;  // slack to align to the 1024-byte swizzle atom
+template <typename T, int BITS, int SLOTS>
+cudaError_t run_bits(const DecodeArgs& a, int rows, int nvt, int cl, cudaStream_t stream) {
+  constexpr int P = 8 / BITS;
+  const size_t smem = ring_smem_bytes<T, SLOTS>() + 1024;  // slack to align to the 1024-byte swizzle atom
   static bool attr_sets[kMaxDevices];  // per device (benign race: every caller sets the same value)
   const int attr_dev = current_device();
   if (attr_dev < 0) return cudaErrorInvalidDevice;
   bool& attr_set = attr_sets[attr_dev];
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_decode_ring<T, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k_decode_ring<T, BITS, SLOTS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(k_decode_ring<T, BITS>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      e = cudaFuncSetAttribute(k_decode_ring<T, BITS, SLOTS>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -540,7 +537,23 @@ cudaError_t run_bits(const DecodeArgs& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_decode_ring<T, BITS>, a, cl, kmap, vmap);
+  return cudaLaunchKernelEx(&cfg, k_decode_ring<T, BITS, SLOTS>, a, cl, kmap, vmap);
+}
+
+template <typename T, int BITS>
+cudaError_t run_bits(const DecodeArgs& a, cudaStream_t stream) {
+  constexpr int kTileTok = 32 * (8 / BITS);
+  const int rows = a.B * a.Hkv;
+  const int nvt = (a.n + kTileTok - 1) / kTileTok;
+  const int per = kSlice / kTileTok;  // V tiles per CTA
+  const int cl = (nvt + per - 1) / per;
+  if (cl > kMaxCl || (long long)rows * cl > 0x7fffffffLL) return cudaErrorNotSupported;
+  if constexpr (BITS >= 4) {
+    return run_bits<T, BITS, 4>(a, rows, nvt, cl, stream);
+  } else {
+    if (ring_slots_2bit((long long)rows * cl, device_sms()) == 4) return run_bits<T, BITS, 4>(a, rows, nvt, cl, stream);
+    return run_bits<T, BITS, 2>(a, rows, nvt, cl, stream);
+  }
 }
 
 template <typename T>

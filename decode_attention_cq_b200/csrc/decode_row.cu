@@ -757,16 +757,6 @@ cudaError_t set_row_attributes(size_t smem) {
   return e;
 }
 
-int device_sms() {
-  static int count[kMaxDevices] = {};  // per device ordinal; 0 until read
-  const int dev = current_device();
-  int c = 0;
-  if (dev < 0) return 0;
-  if (count[dev] == 0 && cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
-    count[dev] = c;
-  return count[dev];
-}
-
 template <typename T>
 cudaError_t run_row(const DecodeArgs& a, cudaStream_t stream) {
   const int rows = a.B * a.Hkv;
