@@ -62,14 +62,13 @@ struct RingFixed {
   float recv[kRecv];                // [src][h][channel - first owned channel]
 };
 
-// Ring slots (SLOTS): 4 with 2 CTAs per SM (more bytes in flight per CTA), or
-// 2 with 3 CTAs per SM (more CTAs resident). 4- and 8-bit codes, where the
-// kernel mostly waits on its copies, always take 4 (8-bit at batch 16,
-// n = 8192: 78.6 -> 67.8 us). 2-bit codes take 4 while the launch fits in two
-// waves of 2 CTAs per SM, 2 beyond that (measured on B200, n = 8192: batch 16
-// 40.9 -> 37.9 us with 4; batch 32 67.4 -> 62.9 us and batch 64 117.2 ->
-// 103.1 us with 2).
-inline int ring_slots_2bit(long long ctas, int sms) { return sms > 0 && ctas <= 4LL * sms ? 4 : 2; }
+// Ring slots (SLOTS): 4 with 2 CTAs per SM (more bytes in flight per CTA)
+// while the launch fits in two waves of 2 CTAs per SM, 2 with 3 CTAs per SM
+// (more CTAs resident) beyond that. Measured on B200 at n = 8192: batch 16
+// takes 4 (2-bit 40.9 -> 37.9 us, 8-bit 78.6 -> 67.8 us); batch 64 takes 2
+// (2-bit 117.2 -> 103.1 us, 4-bit 146.5 -> 129.2 us, 8-bit 211.1 -> 194.6 us);
+// batch 32, 2-bit: 67.4 -> 62.9 us with 2.
+inline int ring_slots_for(long long ctas, int sms) { return sms > 0 && ctas <= 4LL * sms ? 4 : 2; }
 
 // logits / weight fragments (16 B per token) | ring (slots x 16 KB) | fixed part
 template <typename T, int SLOTS>
@@ -548,12 +547,8 @@ cudaError_t run_bits(const DecodeArgs& a, cudaStream_t stream) {
   const int per = kSlice / kTileTok;  // V tiles per CTA
   const int cl = (nvt + per - 1) / per;
   if (cl > kMaxCl || (long long)rows * cl > 0x7fffffffLL) return cudaErrorNotSupported;
-  if constexpr (BITS >= 4) {
-    return run_bits<T, BITS, 4>(a, rows, nvt, cl, stream);
-  } else {
-    if (ring_slots_2bit((long long)rows * cl, device_sms()) == 4) return run_bits<T, BITS, 4>(a, rows, nvt, cl, stream);
-    return run_bits<T, BITS, 2>(a, rows, nvt, cl, stream);
-  }
+  if (ring_slots_for((long long)rows * cl, device_sms()) == 4) return run_bits<T, BITS, 4>(a, rows, nvt, cl, stream);
+  return run_bits<T, BITS, 2>(a, rows, nvt, cl, stream);
 }
 
 template <typename T>

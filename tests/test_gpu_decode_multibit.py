@@ -114,3 +114,28 @@ def test_bitsweep_n8192_batch16_sampled(cuda_device, bits):
     assert torch.all(o >= a - tol) and torch.all(o <= a + s + tol)
     del q, k, v
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_large_launch_two_slot_ring(cuda_device, bits):
+    """A launch past two waves of 2 CTAs per SM (batch 40, n = 8192: 1280
+    CTAs of 2048 tokens) takes the 2-slot ring with 3 CTAs per SM; the first,
+    a middle and the last sequence against the oracle, and every row inside
+    the convex hull alpha_V <= o <= alpha_V + (2^b - 1) s_V."""
+    B, Hkv, n = 40, 8, 8192
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert B * Hkv * 4 > 4 * sms  # the launch this test is for
+    q, k, v = synth.make_case(B, 4 * Hkv, Hkv, n, 128, "f16", outliers=4, seed=900 + bits, device=cuda_device)
+    kq, vq = _quant(k, v, bits, cuda_device)
+    out = cq.cq_decode_attn(q, kq, vq, calib=CALIBS[1])
+    torch.cuda.synchronize()
+    for b in (0, B // 2, B - 1):
+        ref = _ref(q[b:b + 1].cpu(), k[b:b + 1].cpu(), v[b:b + 1].cpu(), bits, CALIBS[1])
+        assert _err(out[b:b + 1], ref, torch.float16) <= OUT_RTOL, b
+    a = vq.alpha.float().repeat_interleave(4, dim=1)
+    s = vq.scale.float().repeat_interleave(4, dim=1) * ((1 << bits) - 1)
+    o = out.float()
+    tol = 1e-3 * (a.abs() + s.abs())
+    assert torch.all(o >= a - tol) and torch.all(o <= a + s + tol)
+    del q, k, v
+    torch.cuda.empty_cache()
